@@ -1,0 +1,431 @@
+#!/usr/bin/env python3
+"""Benchmark of the chunk-causal attention layer on B200.
+
+One step = one pass of the whole layer over one chunk: ``unstep_rope_kv_append`` (3D RoPE +
+ring-buffer KV append) followed by ``unstep_window_attn`` (attention over the window).  The
+default workload is the Wan-1.3B-shaped layer with a full causal cache: 12 heads x 128,
+30x52 = 1560 tokens per latent frame, a chunk of 3 frames (4680 queries) attending all 21 frames
+of a 5-s clip (32760 keys); the cache is filled by streaming chunks 0..6 first, and each timed
+step is a re-forward of the last chunk (the next denoising step).
+
+Output: one JSON line.  ``value`` = attention FLOPs (4*B*H*L*Lk*D, true keys) of all ranks per
+second of step time (device-timed with CUDA events, max over ranks, L2 flushed between steps);
+``e2e`` = the same metric through the public API from pinned host buffers (host->device copy of
+q/k/v and device->host copy of the output inside the timed region).
+
+``--impl reference`` times the fp64 CPU oracle (rank 0 only) on a bounded sample of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "windowed-attn TFLOP/s & chunk-steps/s at Wan-1.3B shape; % bf16/HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------------------------
+# helpers shared with the tests (no GPU needed)
+# ----------------------------------------------------------------------------------------------
+
+def dist_env():
+    """(rank, local_rank, world) from torchrun's environment; (0, 0, 1) when run directly."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank streams its own independent video stream (weak scaling, no exchange)."""
+    return base + 7919 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks of a per-rank time (the job takes as long as its slowest rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:  # noqa: BLE001
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for name in ("window_attn.cu", "sm100.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "causal_video_diffusion_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"window_attn_{workload}.txt")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source:\s*([0-9a-f]+)", text)
+    if not m or m.group(2) != kernel_source_digest():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"unstep_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:  # noqa: BLE001
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, r in rows:
+            for n, flag in zip(names, r[1:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------------
+# the CUDA arm
+# ----------------------------------------------------------------------------------------------
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+    from causal_video_diffusion_b200 import binding
+    from causal_video_diffusion_b200 import workloads as W
+
+    wl = W.WORKLOADS[args.workload]
+    s = wl.shape
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    stream = torch.cuda.current_stream()
+    seed = rank_seed(args.seed, rank)
+    last = wl.chunks - 1
+    F = s.chunk_frames
+    f_last = wl.frame_idx(last)
+    Lk = wl.keys_for_chunk(last)
+    flops = wl.attn_flops(last)
+
+    cache = binding.LayerCache(s.B, s.H, s.D, s.Hg, s.Wg, s.d_t, s.d_h, s.d_w,
+                               cap_frames=wl.cap, max_pos_t=f_last + F, theta=s.theta)
+    # fill the cache: chunks 0 .. last-1, then the last chunk once
+    out = torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16, device=dev)
+    for c in range(wl.chunks):
+        q, k, v = W.gen_qkv(W.qkv_seed(seed, chunk=c), s, device=str(dev))
+        cache.rope_kv_append(q, k, v, wl.frame_idx(c), F)
+        cache.window_attn(q, wl.window, out=out)
+    q_src, k_src, v_src = W.gen_qkv(W.qkv_seed(seed, chunk=last, forward=1), s, device=str(dev))
+    q_work = torch.empty_like(q_src)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    if cache.device_error() != 0:
+        raise RuntimeError("device error during cache fill")
+
+    def one_step(ev):
+        q_work.copy_(q_src)
+        flush.zero_()                       # evict L2 between timed steps
+        ev[0].record(stream)
+        cache.rope_kv_append(q_work, k_src, v_src, f_last, F)   # re-forward of the last chunk
+        ev[1].record(stream)
+        cache.window_attn(q_work, wl.window, out=out)
+        ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        one_step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        one_step(events[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    rope_ms = [e[0].elapsed_time(e[1]) for e in events]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in events]
+    step_ms_local = sum(r + a for r, a in zip(rope_ms, attn_ms)) / args.steps
+    step_ms = reduce_max(step_ms_local, world, dev)
+    err = cache.device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the timed region")
+
+    # e2e through the public API from pinned host buffers
+    q_h = q_src.cpu().pin_memory()
+    k_h = k_src.cpu().pin_memory()
+    v_h = v_src.cpu().pin_memory()
+    out_h = torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16).pin_memory()
+    bufs = {"q": torch.empty_like(q_src), "k": torch.empty_like(k_src),
+            "v": torch.empty_like(v_src), "out": torch.empty_like(out)}
+    e2e_steps = max(1, min(args.steps, 50))
+    for _ in range(3):
+        cache.step_from_host(q_h, k_h, v_h, f_last, F, wl.window, out_h, bufs)
+    torch.cuda.synchronize()
+    e2e_ms_list = []
+    for _ in range(e2e_steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.step_from_host(q_h, k_h, v_h, f_last, F, wl.window, out_h, bufs)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms_list.append(e0.elapsed_time(e1))
+    e2e_ms = reduce_max(sum(e2e_ms_list) / e2e_steps, world, dev)
+
+    peaks, peak_src = load_peaks()
+    attn_avg = reduce_max(sum(attn_ms) / args.steps, world, dev)
+    rope_avg = reduce_max(sum(rope_ms) / args.steps, world, dev)
+    attn_tflops = flops / (attn_avg * 1e-3) / 1e12
+    rope_bytes = wl.rope_bytes()
+    rope_gbs = rope_bytes / (rope_avg * 1e-3) / 1e9
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    act_bytes = s.B * s.L * s.H * s.D * 2
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) fp32 draws rounded to bf16 (q, k, v)",
+        "config": {
+            "workload": f"{wl.name}: B={s.B} H={s.H} D={s.D} grid={s.Hg}x{s.Wg} "
+                        f"L={s.L} keys={Lk} window={wl.window} cap={wl.cap}",
+            "per_rank": "one independent stream per GPU" if world > 1 else "one stream",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+            "parallelism": f"independent streams x{world}",
+        },
+        "chunk_steps_per_s": round(world * s.B / (step_ms * 1e-3), 2),
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": 3 * act_bytes, "d2h_bytes_per_step": act_bytes},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {
+            "kernel": f"window_attn_kernel<{s.D}>",
+            "bound": "tensor",
+            "achieved": round(attn_tflops, 2),
+            "peak": peaks["bf16_tflops"],
+            "peak_source": f"{peak_src} bf16 burst",
+            "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
+            "frac_of_sustained": round(attn_tflops / peaks["bf16_tflops_sustained"], 4),
+            "traffic": profiled_traffic(wl.name),
+            "ms_per_launch": round(attn_avg, 4),
+            "flops_per_launch": flops,
+        },
+        "rope_roofline": {
+            "kernel": f"rope_kv_append_kernel<{s.D}>",
+            "bound": "hbm",
+            "achieved": round(rope_gbs, 1),
+            "peak": peaks["hbm_gbs"],
+            "peak_source": f"{peak_src} copy",
+            "unit": "GB/s",
+            "frac": round(rope_gbs / peaks["hbm_gbs"], 4),
+            "bytes_per_launch": rope_bytes,
+            "us_per_launch": round(rope_avg * 1e3, 2),
+        },
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, q_src, k_src, v_src, cache, args)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------
+# the oracle on the host cores
+# ----------------------------------------------------------------------------------------------
+
+def _oracle_sample(wl, q_bits, k_bits, v_bits, heads, rows_per_head, seed=0):
+    """Time the oracle on a bounded sample of one step: the heads in ``heads`` (RoPE of their q
+    and k over the whole chunk, appended to a cache streamed to the last chunk) and attention for
+    ``rows_per_head`` query rows of each.  Heads are independent and rows cost the same, so the
+    step's time is extrapolated by H/len(heads) for the RoPE and by rows for the attention.
+    Returns (extrapolated step seconds, measured seconds, sample description)."""
+    import numpy as np
+    import oracle
+    s = wl.shape
+    hs = list(heads)
+    qs, ks, vs = (np.ascontiguousarray(a[:, :, hs, :]) for a in (q_bits, k_bits, v_bits))
+    ol = oracle.OracleLayer(s.B, len(hs), s.Hg, s.Wg,
+                            oracle.RopeSpec(s.d_t, s.d_h, s.d_w, s.theta), wl.cap)
+    last = wl.chunks - 1
+    for c in range(last):
+        ol.fill_zero_frames(wl.frame_idx(c), s.chunk_frames)
+    t0 = time.perf_counter()
+    q_rot = ol.append(qs, ks, vs, wl.frame_idx(last), s.chunk_frames)
+    t1 = time.perf_counter()
+    rng = np.random.default_rng(seed)
+    rows = [(b, int(l), h) for b in range(s.B) for h in range(len(hs))
+            for l in rng.choice(s.L, size=min(rows_per_head, s.L), replace=False)]
+    t2 = time.perf_counter()
+    ol.attend(q_rot, wl.window, rows)
+    t3 = time.perf_counter()
+    total_rows = s.B * s.H * s.L
+    step_s = (t1 - t0) * s.H / len(hs) + (t3 - t2) * total_rows / len(rows)
+    sample = (f"RoPE+append of {len(hs)} of {s.H} heads over the whole chunk and fp64 attention "
+              f"of {len(rows)} of {total_rows} query rows, extrapolated to one full step")
+    return step_s, (t1 - t0) + (t3 - t2), sample
+
+
+def cpu_baseline(wl, q, k, v, cache, args):
+    import oracle
+    from causal_video_diffusion_b200 import workloads as W
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_num_threads(cores)
+    qb, kb, vb = (W.bits(t.cpu()) for t in (q, k, v))
+    step_s, measured, sample = _oracle_sample(wl, qb, kb, vb, [0, wl.shape.H - 1], args.cpu_rows)
+    flops = wl.attn_flops(wl.chunks - 1)
+    return {"value": round(flops / step_s / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle", "sample": sample,
+            "seconds_measured": round(measured, 3), "extrapolated_step_s": round(step_s, 3)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from causal_video_diffusion_b200 import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    s = wl.shape
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_num_threads(cores)
+    q, k, v = W.gen_qkv(W.qkv_seed(args.seed, chunk=wl.chunks - 1, forward=1), s)
+    qb, kb, vb = W.bits(q), W.bits(k), W.bits(v)
+    for i in range(args.warmup):
+        _oracle_sample(wl, qb, kb, vb, [i % s.H], args.ref_rows, seed=i)
+    total = 0.0
+    sample = ""
+    for i in range(args.steps):
+        step_s, _, sample = _oracle_sample(wl, qb, kb, vb, [i % s.H], args.ref_rows, seed=i)
+        total += step_s
+    step_s = total / args.steps
+    flops = wl.attn_flops(wl.chunks - 1)
+    value = flops / step_s / 1e12
+    result = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic: seeded N(0,1) bf16",
+        "config": {"workload": f"{wl.name}: B={s.B} H={s.H} D={s.D} grid={s.Hg}x{s.Wg} "
+                               f"L={s.L} keys={wl.keys_for_chunk(wl.chunks - 1)} "
+                               f"window={wl.window} cap={wl.cap}"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                         "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": "per step: " + sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan_full")
+    ap.add_argument("--seed", type=int, default=2024)
+    ap.add_argument("--cpu-rows", type=int, default=1024, help="oracle rows per head (baseline)")
+    ap.add_argument("--ref-rows", type=int, default=32, help="oracle rows per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank, local_rank, world = dist_env()
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, local_rank, world)
+
+
+if __name__ == "__main__":
+    main()

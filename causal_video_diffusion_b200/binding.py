@@ -1,0 +1,268 @@
+"""ctypes binding of ``libunstep.so`` (include/unstep.h).
+
+Argument marshalling only: torch tensors are turned into device pointers and the current CUDA
+stream, shapes are checked against the cache, and every step of the layer runs inside the
+library's kernels.  There is no fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libunstep.so")
+
+UNSTEP_OK = 0
+UNSTEP_ERR_ARG = -1
+UNSTEP_ERR_SHAPE = -2
+UNSTEP_ERR_ALIGN = -3
+UNSTEP_ERR_FRAME_ORDER = -4
+UNSTEP_ERR_WINDOW = -5
+UNSTEP_ERR_UNSUPPORTED = -6
+UNSTEP_ERR_CUDA = -7
+UNSTEP_ERR_DEVICE_TIMEOUT = -8
+
+
+class unstep_cache_t(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int),
+        ("Hg", ctypes.c_int), ("Wg", ctypes.c_int),
+        ("d_t", ctypes.c_int), ("d_h", ctypes.c_int), ("d_w", ctypes.c_int),
+        ("theta", ctypes.c_double),
+        ("cap_frames", ctypes.c_int), ("max_pos_t", ctypes.c_int),
+        ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("slot_frame", ctypes.c_void_p), ("cos_sin", ctypes.c_void_p),
+        ("dev_error", ctypes.c_void_p),
+        ("frames_written", ctypes.c_int), ("first_frame", ctypes.c_int),
+        ("last_chunk_start", ctypes.c_int), ("last_chunk_frames", ctypes.c_int),
+        ("initialized", ctypes.c_int),
+    ]
+
+
+class unstep_grid_t(ctypes.Structure):
+    _fields_ = [("frames", ctypes.c_int), ("Hg", ctypes.c_int), ("Wg", ctypes.c_int)]
+
+
+class unstep_window_plan_t(ctypes.Structure):
+    _fields_ = [("first_frame", ctypes.c_int), ("last_frame", ctypes.c_int),
+                ("keys", ctypes.c_int), ("seg_row", ctypes.c_int * 2),
+                ("seg_len", ctypes.c_int * 2)]
+
+
+# every symbol include/unstep.h declares, with its ctypes signature
+_SIGNATURES = {
+    "unstep_version": ([], ctypes.c_int),
+    "unstep_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "unstep_cache_table_bytes": ([ctypes.POINTER(unstep_cache_t)], ctypes.c_size_t),
+    "unstep_cache_kv_bytes": ([ctypes.POINTER(unstep_cache_t)], ctypes.c_size_t),
+    "unstep_cache_init": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
+    "unstep_append_plan": ([ctypes.POINTER(unstep_cache_t), ctypes.c_int, unstep_grid_t,
+                            ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+    "unstep_rope_kv_append": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                               ctypes.POINTER(unstep_cache_t), ctypes.c_int, unstep_grid_t,
+                               ctypes.c_void_p], ctypes.c_int),
+    "unstep_window_plan": ([ctypes.POINTER(unstep_cache_t), ctypes.c_int,
+                            ctypes.POINTER(unstep_window_plan_t)], ctypes.c_int),
+    "unstep_window_attn": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t), ctypes.c_int,
+                            ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
+    "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
+                                     ctypes.c_int),
+}
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+class UnstepError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})" if what else
+                         f"{status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libunstep.so; raises if it is missing (build it with causal_video_diffusion_b200.build)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: the CUDA library has not been built "
+                               "(python -m causal_video_diffusion_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def status_string(rc: int) -> str:
+    try:
+        return lib().unstep_status_string(int(rc)).decode()
+    except Exception:  # noqa: BLE001 - used while formatting an error
+        return "status"
+
+
+def _check(rc: int, what: str) -> int:
+    if rc < 0:
+        raise UnstepError(rc, what)
+    return rc
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return int(t.data_ptr())
+
+
+class LayerCache:
+    """One attention layer's ring-buffer KV cache and RoPE tables, in caller-owned torch memory.
+
+    All device memory is allocated here by torch; the library only reads and writes it.
+    """
+
+    def __init__(self, B: int, H: int, D: int, Hg: int, Wg: int, d_t: int, d_h: int, d_w: int,
+                 cap_frames: int, max_pos_t: int, theta: float = 10000.0,
+                 device: Optional[torch.device] = None,
+                 stream: Optional[torch.cuda.Stream] = None):
+        L = lib()
+        dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                           torch.cuda.current_device())
+        c = unstep_cache_t()
+        c.B, c.H, c.D, c.Hg, c.Wg = B, H, D, Hg, Wg
+        c.d_t, c.d_h, c.d_w, c.theta = d_t, d_h, d_w, float(theta)
+        c.cap_frames, c.max_pos_t = cap_frames, max_pos_t
+        tab_bytes = L.unstep_cache_table_bytes(ctypes.byref(c))
+        if tab_bytes == 0:
+            raise UnstepError(UNSTEP_ERR_ARG, "cache shape rejected")
+        self.Tf = Hg * Wg
+        self.rows = cap_frames * self.Tf
+        self.k_cache = torch.empty((B, H, self.rows, D), dtype=torch.bfloat16, device=dev)
+        self.v_cache = torch.empty_like(self.k_cache)
+        self.slot_frame = torch.empty((cap_frames,), dtype=torch.int32, device=dev)
+        self.cos_sin = torch.empty((tab_bytes // 4,), dtype=torch.float32, device=dev)
+        self.dev_error = torch.zeros((1,), dtype=torch.int32, device=dev)
+        c.k_cache = self.k_cache.data_ptr()
+        c.v_cache = self.v_cache.data_ptr()
+        c.slot_frame = self.slot_frame.data_ptr()
+        c.cos_sin = self.cos_sin.data_ptr()
+        c.dev_error = self.dev_error.data_ptr()
+        self.c = c
+        self.device = dev
+        with torch.cuda.device(dev):
+            _check(L.unstep_cache_init(ctypes.byref(c), _stream_handle(stream)),
+                   "unstep_cache_init")
+
+    # -- metadata ---------------------------------------------------------------------------
+    @property
+    def shape(self):
+        c = self.c
+        return c.B, c.H, c.D
+
+    @property
+    def frames_written(self) -> int:
+        return self.c.frames_written
+
+    @property
+    def last_chunk(self):
+        return self.c.last_chunk_start, self.c.last_chunk_frames
+
+    def chunk_len(self, frames: int) -> int:
+        return frames * self.Tf
+
+    def _check_act(self, t: torch.Tensor, L: int, name: str):
+        c = self.c
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bfloat16")
+        if tuple(t.shape) != (c.B, L, c.H, c.D):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(c.B, L, c.H, c.D)}")
+        if t.device != self.device:
+            raise ValueError(f"{name} is on {t.device}, the cache on {self.device}")
+
+    # -- the library calls ------------------------------------------------------------------
+    def append_plan(self, frame_idx: int, frames: int):
+        slots = (ctypes.c_int * max(1, frames))()
+        g = unstep_grid_t(frames, self.c.Hg, self.c.Wg)
+        rc = lib().unstep_append_plan(ctypes.byref(self.c), int(frame_idx), g, slots)
+        _check(rc, "unstep_append_plan")
+        return bool(rc), list(slots)[:frames]
+
+    def window_plan(self, window: int) -> unstep_window_plan_t:
+        plan = unstep_window_plan_t()
+        _check(lib().unstep_window_plan(ctypes.byref(self.c), int(window), ctypes.byref(plan)),
+               "unstep_window_plan")
+        return plan
+
+    def rope_kv_append(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       frame_idx: int, frames: int,
+                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Rotate q in place, append rotated k and v to the ring; returns q."""
+        L = self.chunk_len(frames)
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_act(t, L, n)
+        g = unstep_grid_t(frames, self.c.Hg, self.c.Wg)
+        rc = lib().unstep_rope_kv_append(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                         ctypes.byref(self.c), int(frame_idx), g,
+                                         _stream_handle(stream))
+        _check(rc, "unstep_rope_kv_append")
+        return q
+
+    def window_attn(self, q: torch.Tensor, window: int, out: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Attention of the latest chunk's rotated queries over the last ``window`` frames."""
+        L = self.chunk_len(self.c.last_chunk_frames)
+        self._check_act(q, L, "q")
+        if out is None:
+            out = torch.empty_like(q)
+        self._check_act(out, L, "out")
+        rc = lib().unstep_window_attn(_dev_ptr(q, "q"), ctypes.byref(self.c), int(window),
+                                      _dev_ptr(out, "out"), _stream_handle(stream))
+        _check(rc, "unstep_window_attn")
+        return out
+
+    def device_error(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        return lib().unstep_get_device_error(ctypes.byref(self.c), _stream_handle(stream))
+
+    def step_from_host(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor,
+                       frame_idx: int, frames: int, window: int, out_h: torch.Tensor,
+                       bufs: dict, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """One layer step from pinned host tensors: copy in, append, attend, copy out.
+
+        ``bufs`` holds the device staging tensors ``q``, ``k``, ``v``, ``out`` (reused).
+        The copies and both calls are enqueued on the stream; ``out_h`` is valid after a sync.
+        """
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            bufs["q"].copy_(q_h, non_blocking=True)
+            bufs["k"].copy_(k_h, non_blocking=True)
+            bufs["v"].copy_(v_h, non_blocking=True)
+            self.rope_kv_append(bufs["q"], bufs["k"], bufs["v"], frame_idx, frames, stream=s)
+            self.window_attn(bufs["q"], window, out=bufs["out"], stream=s)
+            out_h.copy_(bufs["out"], non_blocking=True)
+        return out_h
+
+
+def selftest_wait_timeout(dev_error: torch.Tensor, limit_ns: int,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    _check(lib().unstep_selftest_wait_timeout(_dev_ptr(dev_error, "dev_error"), int(limit_ns),
+                                              _stream_handle(stream)),
+           "unstep_selftest_wait_timeout")
+
+
+def declared_symbols(header: Optional[str] = None):
+    """Function names declared in include/unstep.h (parsed from the header text)."""
+    import re
+    header = header or os.path.join(os.path.dirname(_HERE), "include", "unstep.h")
+    text = open(header).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s*(unstep_[a-z_0-9]+)\s*\(",
+                                 text, flags=re.M)))

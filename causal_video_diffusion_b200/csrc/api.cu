@@ -1,0 +1,343 @@
+// api.cu -- host side of the C ABI declared in include/unstep.h: argument validation, cache
+// metadata, the RoPE coefficient tables, window resolution, TMA descriptors and launches.
+//
+// UnStep paper (arXiv 2609.32518), abstract: RoPE "with cached coefficients", KV indexing and a
+// limited temporal window of the attention KV cache; Table 3: chunks of three latent frames.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "../../include/unstep.h"
+#include "internal.h"
+
+namespace {
+
+constexpr int kInitMagic = 0x55535450;  // "USTP"
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape fields only (no pointers): 0 if valid, else a status code.
+int check_shape(const unstep_cache_t *c) {
+  if (!c) return UNSTEP_ERR_ARG;
+  if (c->B < 1 || c->H < 1 || c->Hg < 1 || c->Wg < 1 || c->cap_frames < 1 || c->max_pos_t < 1)
+    return UNSTEP_ERR_ARG;
+  if (c->d_t < 0 || c->d_h < 0 || c->d_w < 0 || (c->d_t & 1) || (c->d_h & 1) || (c->d_w & 1))
+    return UNSTEP_ERR_ARG;
+  if (c->d_t + c->d_h + c->d_w != c->D) return UNSTEP_ERR_ARG;
+  if (!(c->theta > 0.0) || !std::isfinite(c->theta)) return UNSTEP_ERR_ARG;
+  if (c->D != 64 && c->D != 128) return UNSTEP_ERR_UNSUPPORTED;
+  // row and element indices of the kernels: rows per (b, h) and TMA extents fit in int32,
+  // every element offset in int64
+  const long long tf = static_cast<long long>(c->Hg) * c->Wg;
+  const long long rows = tf * c->cap_frames;
+  if (tf > (1ll << 24) || rows > (1ll << 30) || static_cast<long long>(c->B) * c->H > (1ll << 30))
+    return UNSTEP_ERR_UNSUPPORTED;
+  if (c->max_pos_t > (1 << 24)) return UNSTEP_ERR_UNSUPPORTED;
+  return UNSTEP_OK;
+}
+
+size_t table_floats(const unstep_cache_t *c) {
+  return 2ull * (static_cast<size_t>(c->max_pos_t) * (c->d_t / 2) +
+                 static_cast<size_t>(c->Hg) * (c->d_h / 2) +
+                 static_cast<size_t>(c->Wg) * (c->d_w / 2));
+}
+
+int check_ready(const unstep_cache_t *c) {
+  int rc = check_shape(c);
+  if (rc) return rc;
+  if (c->initialized != kInitMagic) return UNSTEP_ERR_ARG;
+  if (!c->k_cache || !c->v_cache || !c->slot_frame || !c->cos_sin || !c->dev_error)
+    return UNSTEP_ERR_ARG;
+  return UNSTEP_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, fetched once through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle: dims[0] is the contiguous channel axis (boxed 64 wide).
+bool encode_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                 const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                  const_cast<void *>(base), dims, strides_bytes, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+int unstep_version(void) { return 100; }
+
+const char *unstep_status_string(int status) {
+  switch (status) {
+    case UNSTEP_OK: return "ok";
+    case UNSTEP_ERR_ARG: return "invalid argument";
+    case UNSTEP_ERR_SHAPE: return "shape mismatch";
+    case UNSTEP_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case UNSTEP_ERR_FRAME_ORDER: return "frame_idx is neither the next chunk nor the latest chunk";
+    case UNSTEP_ERR_WINDOW: return "window outside [chunk frames, cache capacity] or empty cache";
+    case UNSTEP_ERR_UNSUPPORTED: return "unsupported head width or size";
+    case UNSTEP_ERR_CUDA: return "CUDA runtime error";
+    case UNSTEP_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t unstep_cache_table_bytes(const unstep_cache_t *cache) {
+  if (check_shape(cache)) return 0;
+  return table_floats(cache) * sizeof(float);
+}
+
+size_t unstep_cache_kv_bytes(const unstep_cache_t *cache) {
+  if (check_shape(cache)) return 0;
+  return static_cast<size_t>(cache->B) * cache->H * cache->cap_frames * cache->Hg * cache->Wg *
+         cache->D * 2;
+}
+
+int unstep_cache_init(unstep_cache_t *cache, unstep_stream_t stream) {
+  int rc = check_shape(cache);
+  if (rc) return rc;
+  if (!cache->k_cache || !cache->v_cache || !cache->slot_frame || !cache->cos_sin ||
+      !cache->dev_error)
+    return UNSTEP_ERR_ARG;
+  if (!aligned16(cache->k_cache) || !aligned16(cache->v_cache) || !aligned16(cache->cos_sin))
+    return UNSTEP_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // cached coefficients: cos/sin of pos * theta^(-2j/d_a), computed in fp64, stored fp32
+  std::vector<float> tab(table_floats(cache));
+  size_t o = 0;
+  const int dims[3] = {cache->d_t, cache->d_h, cache->d_w};
+  const int npos[3] = {cache->max_pos_t, cache->Hg, cache->Wg};
+  for (int a = 0; a < 3; ++a) {
+    const int half = dims[a] / 2;
+    for (int pos = 0; pos < npos[a]; ++pos) {
+      for (int j = 0; j < half; ++j) {
+        const double inv = std::pow(cache->theta, -2.0 * j / static_cast<double>(dims[a]));
+        const double ang = static_cast<double>(pos) * inv;
+        tab[o++] = static_cast<float>(std::cos(ang));
+        tab[o++] = static_cast<float>(std::sin(ang));
+      }
+    }
+  }
+  const size_t kvb = unstep_cache_kv_bytes(cache);
+  if (cudaMemcpyAsync(cache->cos_sin, tab.data(), tab.size() * sizeof(float),
+                      cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemsetAsync(cache->k_cache, 0, kvb, s) != cudaSuccess ||
+      cudaMemsetAsync(cache->v_cache, 0, kvb, s) != cudaSuccess ||
+      cudaMemsetAsync(cache->slot_frame, 0xFF, sizeof(int) * cache->cap_frames, s) !=
+          cudaSuccess ||
+      cudaMemsetAsync(cache->dev_error, 0, sizeof(int), s) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  cache->frames_written = 0;
+  cache->first_frame = 0;
+  cache->last_chunk_start = -1;
+  cache->last_chunk_frames = 0;
+  cache->initialized = kInitMagic;
+  return UNSTEP_OK;
+}
+
+int unstep_append_plan(const unstep_cache_t *cache, int frame_idx, unstep_grid_t grid,
+                       int *slots_out) {
+  int rc = check_shape(cache);
+  if (rc) return rc;
+  if (cache->initialized != kInitMagic) return UNSTEP_ERR_ARG;
+  if (grid.Hg != cache->Hg || grid.Wg != cache->Wg || grid.frames < 1) return UNSTEP_ERR_SHAPE;
+  if (grid.frames > cache->cap_frames) return UNSTEP_ERR_WINDOW;
+  if (frame_idx < 0 || static_cast<long long>(frame_idx) + grid.frames > cache->max_pos_t)
+    return UNSTEP_ERR_ARG;
+  int is_new;
+  if (cache->last_chunk_frames == 0) {
+    is_new = 1;  // the stream's first chunk may start at any temporal position
+  } else if (frame_idx == cache->frames_written) {
+    is_new = 1;
+  } else if (frame_idx == cache->last_chunk_start && grid.frames == cache->last_chunk_frames) {
+    is_new = 0;
+  } else {
+    return UNSTEP_ERR_FRAME_ORDER;
+  }
+  if (slots_out)
+    for (int i = 0; i < grid.frames; ++i) slots_out[i] = (frame_idx + i) % cache->cap_frames;
+  return is_new;
+}
+
+int unstep_rope_kv_append(void *q, const void *k, const void *v, unstep_cache_t *cache,
+                          int frame_idx, unstep_grid_t grid, unstep_stream_t stream) {
+  int rc = check_ready(cache);
+  if (rc) return rc;
+  if (!q || !k || !v) return UNSTEP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return UNSTEP_ERR_ALIGN;
+  const int is_new = unstep_append_plan(cache, frame_idx, grid, nullptr);
+  if (is_new < 0) return is_new;
+  unstep::RopeAppendParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.k_cache = cache->k_cache;
+  p.v_cache = cache->v_cache;
+  p.slot_frame = cache->slot_frame;
+  const float2 *tab = reinterpret_cast<const float2 *>(cache->cos_sin);
+  p.tab_t = tab;
+  p.tab_h = p.tab_t + static_cast<size_t>(cache->max_pos_t) * (cache->d_t / 2);
+  p.tab_w = p.tab_h + static_cast<size_t>(cache->Hg) * (cache->d_h / 2);
+  p.B = cache->B;
+  p.H = cache->H;
+  p.D = cache->D;
+  p.Hg = cache->Hg;
+  p.Wg = cache->Wg;
+  p.Tf = cache->Hg * cache->Wg;
+  p.L = grid.frames * p.Tf;
+  p.half_t = cache->d_t / 2;
+  p.half_h = cache->d_h / 2;
+  p.half_w = cache->d_w / 2;
+  p.frame_idx = frame_idx;
+  p.frames = grid.frames;
+  p.cap = cache->cap_frames;
+  p.rows = cache->cap_frames * p.Tf;
+  if (unstep::launch_rope_kv_append(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  if (is_new) {
+    if (cache->last_chunk_frames == 0) cache->first_frame = frame_idx;
+    cache->frames_written = frame_idx + grid.frames;
+  }
+  cache->last_chunk_start = frame_idx;
+  cache->last_chunk_frames = grid.frames;
+  return UNSTEP_OK;
+}
+
+int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_plan_t *plan) {
+  int rc = check_shape(cache);
+  if (rc) return rc;
+  if (!plan || cache->initialized != kInitMagic) return UNSTEP_ERR_ARG;
+  if (cache->last_chunk_frames < 1) return UNSTEP_ERR_WINDOW;
+  if (window < cache->last_chunk_frames || window > cache->cap_frames) return UNSTEP_ERR_WINDOW;
+  const int tf = cache->Hg * cache->Wg;
+  const int cap = cache->cap_frames;
+  const int f_end = cache->last_chunk_start + cache->last_chunk_frames - 1;
+  int f0 = f_end - window + 1;
+  if (f0 < cache->first_frame) f0 = cache->first_frame;
+  const int nf = f_end - f0 + 1;
+  const int s0 = f0 % cap;
+  plan->first_frame = f0;
+  plan->last_frame = f_end;
+  plan->keys = nf * tf;
+  plan->seg_row[0] = s0 * tf;
+  if (s0 + nf <= cap) {
+    plan->seg_len[0] = nf * tf;
+    plan->seg_row[1] = 0;
+    plan->seg_len[1] = 0;
+  } else {
+    plan->seg_len[0] = (cap - s0) * tf;
+    plan->seg_row[1] = 0;
+    plan->seg_len[1] = (s0 + nf - cap) * tf;
+  }
+  return UNSTEP_OK;
+}
+
+int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
+                       unstep_stream_t stream) {
+  int rc = check_ready(cache);
+  if (rc) return rc;
+  if (!q || !out) return UNSTEP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(out)) return UNSTEP_ERR_ALIGN;
+  unstep_window_plan_t plan;
+  rc = unstep_window_plan(cache, window, &plan);
+  if (rc) return rc;
+  const int D = cache->D, H = cache->H, B = cache->B;
+  const int tf = cache->Hg * cache->Wg;
+  const int L = cache->last_chunk_frames * tf;
+  const long long R = static_cast<long long>(cache->cap_frames) * tf;
+
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+    const cuuint64_t str[3] = {static_cast<cuuint64_t>(D) * 2,
+                               static_cast<cuuint64_t>(H) * D * 2,
+                               static_cast<cuuint64_t>(L) * H * D * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (!encode_bf16(&tq, q, 4, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(R),
+                                static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t str[2] = {static_cast<cuuint64_t>(D) * 2,
+                               static_cast<cuuint64_t>(R) * D * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!encode_bf16(&tk, cache->k_cache, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
+    if (!encode_bf16(&tv, cache->v_cache, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  unstep::AttnParams p{};
+  p.out = out;
+  p.dev_error = cache->dev_error;
+  p.B = B;
+  p.H = H;
+  p.L = L;
+  p.n_pairs = (L + 255) / 256;
+  for (int s = 0; s < 2; ++s) {
+    p.seg_row[s] = plan.seg_row[s];
+    p.seg_len[s] = plan.seg_len[s];
+    p.seg_tiles[s] = (plan.seg_len[s] + 127) / 128;
+  }
+  p.n_tiles = p.seg_tiles[0] + p.seg_tiles[1];
+  p.scale_log2 = static_cast<float>(1.4426950408889634073599 / std::sqrt(static_cast<double>(D)));
+  p.wait_limit_ns = unstep::kWaitLimitNs;
+  if (unstep::launch_window_attn(D, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
+int unstep_get_device_error(const unstep_cache_t *cache, unstep_stream_t stream) {
+  if (!cache || !cache->dev_error) return UNSTEP_ERR_ARG;
+  int v = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, cache->dev_error, sizeof(int), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return v;
+}
+
+int unstep_selftest_wait_timeout(int *dev_error, uint64_t limit_ns, unstep_stream_t stream) {
+  if (!dev_error) return UNSTEP_ERR_ARG;
+  if (unstep::launch_wait_timeout_selftest(dev_error, limit_ns,
+                                           reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
+}  // extern "C"

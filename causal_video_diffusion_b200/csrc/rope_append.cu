@@ -1,0 +1,145 @@
+// rope_append.cu -- fused 3D RoPE + ring-buffer KV-cache append (one launch per chunk).
+//
+// UnStep paper (arXiv 2609.32518), abstract: the DiT runtime stack applies RoPE from cached
+// coefficients and indexes a KV cache that retains a limited temporal window.  This kernel does
+// both in one pass over HBM: q, k, v are read once; rotated q goes back in place, rotated k and v
+// go to ring slot f mod cap.  The work is pure streaming (6 bf16 tensors of B*L*H*D elements),
+// so it is bound by HBM bandwidth: every thread moves 16-byte vectors, a warp covers 512
+// contiguous bytes of each input, and the coefficient tables (< 20 KB) stay in L1/L2.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace unstep {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kItemsPerThread = 2;  // independent 16-byte vectors in flight per thread
+
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint4 ld_plain(const void *p) {
+  return *reinterpret_cast<const uint4 *>(p);
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_rn(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Rotate one packed bf16 pair (a = low, b = high) by (c, s): (a c - b s, a s + b c).
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float2 cs) {
+  const float a = bf_lo(w), b = bf_hi(w);
+  const float ra = fmaf(a, cs.x, -b * cs.y);
+  const float rb = fmaf(a, cs.y, b * cs.x);
+  return pack_rn(ra, rb);
+}
+
+struct Item {
+  long long e;       // element offset of the 8-channel vector in q/k/v
+  long long ce;      // element offset in the caches
+  float2 cs[4];      // cos/sin of its 4 channel pairs
+};
+
+template <int D>
+__device__ __forceinline__ void locate(const RopeAppendParams &p, long long it, Item &m) {
+  constexpr int V = D / 8;  // 16-byte vectors per head row
+  const int c8 = static_cast<int>(it % V);
+  const long long r = it / V;  // (b*L + l)*H + h
+  const int h = static_cast<int>(r % p.H);
+  const long long bl = r / p.H;
+  const int l = static_cast<int>(bl % p.L);
+  const int b = static_cast<int>(bl / p.L);
+  const int i = l / p.Tf;
+  const int tok = l - i * p.Tf;
+  const int y = tok / p.Wg;
+  const int x = tok - y * p.Wg;
+  const int f = p.frame_idx + i;
+  const int slot = f % p.cap;
+  m.e = it * 8;
+  m.ce = ((static_cast<long long>(b) * p.H + h) * p.rows + static_cast<long long>(slot) * p.Tf +
+          tok) * D + c8 * 8;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int pr = c8 * 4 + u;  // channel pair index
+    const float2 *src;
+    if (pr < p.half_t) {
+      src = p.tab_t + static_cast<long long>(f) * p.half_t + pr;
+    } else if (pr < p.half_t + p.half_h) {
+      src = p.tab_h + y * p.half_h + (pr - p.half_t);
+    } else {
+      src = p.tab_w + x * p.half_w + (pr - p.half_t - p.half_h);
+    }
+    m.cs[u] = __ldg(src);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppendParams p,
+                                                                   long long n_items) {
+  const long long base =
+      static_cast<long long>(blockIdx.x) * (kThreads * kItemsPerThread) + threadIdx.x;
+  if (blockIdx.x == 0 && threadIdx.x < p.frames) {
+    const int f = p.frame_idx + threadIdx.x;
+    p.slot_frame[f % p.cap] = f;
+  }
+  Item m[kItemsPerThread];
+  uint4 qv[kItemsPerThread], kv[kItemsPerThread], vv[kItemsPerThread];
+  bool live[kItemsPerThread];
+#pragma unroll
+  for (int u = 0; u < kItemsPerThread; ++u) {
+    const long long it = base + u * kThreads;
+    live[u] = it < n_items;
+    if (live[u]) {
+      locate<D>(p, it, m[u]);
+      qv[u] = ld_plain(static_cast<const __nv_bfloat16 *>(p.q) + m[u].e);
+      kv[u] = ld_stream(static_cast<const __nv_bfloat16 *>(p.k) + m[u].e);
+      vv[u] = ld_stream(static_cast<const __nv_bfloat16 *>(p.v) + m[u].e);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kItemsPerThread; ++u) {
+    if (!live[u]) continue;
+    uint4 qo, ko;
+    qo.x = rotate_pair(qv[u].x, m[u].cs[0]);
+    qo.y = rotate_pair(qv[u].y, m[u].cs[1]);
+    qo.z = rotate_pair(qv[u].z, m[u].cs[2]);
+    qo.w = rotate_pair(qv[u].w, m[u].cs[3]);
+    ko.x = rotate_pair(kv[u].x, m[u].cs[0]);
+    ko.y = rotate_pair(kv[u].y, m[u].cs[1]);
+    ko.z = rotate_pair(kv[u].z, m[u].cs[2]);
+    ko.w = rotate_pair(kv[u].w, m[u].cs[3]);
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.q) + m[u].e) = qo;
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.k_cache) + m[u].ce) = ko;
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.v_cache) + m[u].ce) = vv[u];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream) {
+  const long long n_items = static_cast<long long>(p.B) * p.L * p.H * (p.D / 8);
+  const long long per_block = kThreads * kItemsPerThread;
+  long long blocks = (n_items + per_block - 1) / per_block;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  if (p.D == 128) {
+    rope_kv_append_kernel<128><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(p, n_items);
+  } else if (p.D == 64) {
+    rope_kv_append_kernel<64><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(p, n_items);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace unstep

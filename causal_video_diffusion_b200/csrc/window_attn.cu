@@ -1,0 +1,415 @@
+// window_attn.cu -- windowed chunk-causal attention on the Blackwell tensor cores.
+//
+// UnStep paper (arXiv 2609.32518): the chunk's queries attend to the keys of the limited
+// temporal window kept in the KV cache (abstract; Table 1 row C4), all queries of a chunk seeing
+// the same key set.  out = softmax(q K^T / sqrt(D)) V, computed as a streaming (online) softmax
+// over 128-key tiles:
+//
+//   S_j  = Q K_j^T                      tcgen05.mma, A = Q (smem), B = K_j (smem), fp32 in TMEM
+//   m    = running max (raised lazily), P_j = exp2(S_j * log2(e)/sqrt(D) - m)   (fp32 -> bf16)
+//   O   += P_j V_j                      tcgen05.mma, A = P_j (TMEM, aliasing S_j), B = V_j (smem)
+//   l   += rowsum(P_j);   out = O / l  (bf16)
+//
+// Work split of one CTA (one (stream, head) and two 128-row query tiles, 320 threads):
+//   warps 0-3  softmax + epilogue of query tile 0 (thread t owns TMEM lane / query row t)
+//   warps 4-7  softmax + epilogue of query tile 1
+//   warp  8    TMA producer: Q once, then K_0, V_0, K_1, V_1, ... through an NS-stage ring
+//   warp  9    MMA issuer (one thread): QK^T and PV for both tiles, ping-ponging so that the
+//              tensor core works on one tile while the other tile's softmax runs
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+//
+// The ring cache holds the window as at most two contiguous row ranges; each range is tiled on
+// its own (its last tile masked), so a tile never straddles the wrap and the ring slot offset is
+// simply the TMA row coordinate.  The running max is only raised when a tile's max exceeds it
+// by more than 8 (log2 units): below that, P <= 2^8 is exact enough in bf16/fp32 and O needs no
+// rescale; above it, the owning warp rescales its O rows in TMEM after the previous PV retired.
+//
+// Every wait is bounded (WaitGuard): on a timeout the CTA records UNSTEP_ERR_DEVICE_TIMEOUT,
+// lets in-flight TMA copies and MMAs land, frees TMEM and exits.
+#include <cuda_bf16.h>
+
+#include "../../include/unstep.h"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace unstep {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+template <int D>
+struct Cfg {
+  static constexpr int kBoxes = D / 64;                // 128-byte swizzle boxes per row
+  static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16
+  static constexpr int kStages = 4;                    // K/V ring stages
+  static constexpr int kSmemQ = 0;
+  static constexpr int kSmemKV = 2 * kTileBytes;
+  static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
+  static constexpr int kSmemUsed = kSmemBar + 256;
+  // at least ~116 KB so that a second CTA (which would block on TMEM) never shares the SM
+  static constexpr int kSmemAlloc = (kSmemUsed + 1024 > 118 * 1024) ? kSmemUsed + 1024
+                                                                    : 118 * 1024;
+  static constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO0 = 256, kTmO1 = 256 + D;
+  static constexpr uint32_t kTmCols = 512;
+};
+
+__device__ __forceinline__ void key_tile(const AttnParams &p, int t, int &row, int &valid) {
+  if (t < p.seg_tiles[0]) {
+    row = p.seg_row[0] + t * 128;
+    valid = min(128, p.seg_len[0] - t * 128);
+  } else {
+    const int u = t - p.seg_tiles[0];
+    row = p.seg_row[1] + u * 128;
+    valid = min(128, p.seg_len[1] - u * 128);
+  }
+}
+
+// A wait used only while tearing down after an abort: ignores the abort flag.
+__device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    window_attn_kernel(const __grid_constant__ CUtensorMap tmq,
+                       const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
+  using C = Cfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kSmemBar);
+  uint64_t *q_full = bars;
+  uint64_t *full = bars + 1;
+  uint64_t *empty = full + NS;
+  uint64_t *s_full = empty + NS;
+  uint64_t *p_ready = s_full + 2;
+  uint64_t *o_done = p_ready + 2;
+  uint64_t *drain = o_done + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x % p.n_pairs;
+  const int bh = blockIdx.x / p.n_pairs;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+  const int q0 = pair * 256;
+  const bool has1 = q0 + 128 < p.L;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_ready[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, C::kTmCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard g{abort_flag, p.dev_error, p.wait_limit_ns};
+  constexpr int E = UNSTEP_ERR_DEVICE_TIMEOUT;
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmq);
+      tma_prefetch_desc(&tmk);
+      tma_prefetch_desc(&tmv);
+      const int nq = has1 ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * C::kTileBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int c = 0; c < C::kBoxes; ++c)
+          tma_load_4d(smem + C::kSmemQ + t * C::kTileBytes + c * 16384, &tmq, q_full, c * 64, h,
+                      q0 + t * 128, b);
+      const int n_loads = 2 * p.n_tiles;
+      int issued = 0;
+      for (int n = 0; n < n_loads; ++n) {
+        const int s = n % NS;
+        const uint32_t r = static_cast<uint32_t>(n / NS);
+        if (!wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E)) break;
+        mbar_arrive_expect_tx(&full[s], C::kTileBytes);
+        int row, valid;
+        key_tile(p, n >> 1, row, valid);
+        const CUtensorMap *m = (n & 1) ? &tmv : &tmk;
+        for (int c = 0; c < C::kBoxes; ++c)
+          tma_load_3d(smem + C::kSmemKV + s * C::kTileBytes + c * 16384, m, &full[s], c * 64,
+                      row, bh);
+        issued = n + 1;
+      }
+      if (*abort_flag) {
+        // let every copy still in flight land before the CTA's shared memory is released
+        for (int n = max(0, issued - NS); n < issued; ++n)
+          wait_drain(&full[n % NS], static_cast<uint32_t>(n / NS) & 1u);
+        wait_drain(q_full, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
+      const uint32_t sQ = smem_u32(smem + C::kSmemQ);
+      const uint32_t sKV = smem_u32(smem + C::kSmemKV);
+      auto qk = [&](int t, int s) {
+        const uint32_t dS = tmem + (t ? C::kTmS1 : C::kTmS0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
+          const uint64_t a = sdesc_sw128(sQ + t * C::kTileBytes + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sKV + s * C::kTileBytes + off, 16, 1024);
+          umma_ss(dS, a, bd, kIdQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto pv = [&](int t, int s, bool acc) {
+        const uint32_t dO = tmem + (t ? C::kTmO1 : C::kTmO0);
+        const uint32_t aP = tmem + (t ? C::kTmS1 : C::kTmS0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc_sw128(sKV + s * C::kTileBytes + kk * 2048, 16384, 1024);
+          umma_ts(dO, aP + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_full = [&](int n) {
+        return wait_bounded(&full[n % NS], static_cast<uint32_t>(n / NS) & 1u, g, E);
+      };
+      bool ok = wait_bounded(q_full, 0, g, E) && wait_full(0);
+      if (ok) {
+        tc_fence_after();
+        qk(0, 0);
+        umma_commit(&s_full[0]);
+        if (has1) {
+          qk(1, 0);
+          umma_commit(&s_full[1]);
+        }
+        umma_commit(&empty[0]);
+      }
+      for (int j = 0; ok && j < p.n_tiles; ++j) {
+        const int nv = 2 * j + 1, nk = 2 * j + 2;
+        const int sv = nv % NS, sk = nk % NS;
+        const bool more = j + 1 < p.n_tiles;
+        const uint32_t ph = static_cast<uint32_t>(j) & 1u;
+        if (!(ok = wait_full(nv))) break;
+        if (!(ok = wait_bounded(&p_ready[0], ph, g, E))) break;
+        tc_fence_after();
+        pv(0, sv, j > 0);
+        umma_commit(&o_done[0]);
+        if (more) {
+          if (!(ok = wait_full(nk))) break;
+          tc_fence_after();
+          qk(0, sk);
+          umma_commit(&s_full[0]);
+        }
+        if (has1) {
+          if (!(ok = wait_bounded(&p_ready[1], ph, g, E))) break;
+          tc_fence_after();
+          pv(1, sv, j > 0);
+          umma_commit(&o_done[1]);
+        }
+        umma_commit(&empty[sv]);
+        if (more) {
+          if (has1) {
+            qk(1, sk);
+            umma_commit(&s_full[1]);
+          }
+          umma_commit(&empty[sk]);
+        }
+      }
+      // every MMA issued above has completed once `drain` flips
+      umma_commit(drain);
+      wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- softmax + epilogue
+    const int i = warp >> 2;          // query tile of this warpgroup
+    const int wq = warp & 3;          // TMEM lane quarter
+    const int row = threadIdx.x & 127;
+    if (i == 0 || has1) {
+      const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_base + (i ? C::kTmS1 : C::kTmS0);
+      const uint32_t tO = tmem + lane_base + (i ? C::kTmO1 : C::kTmO0);
+      const float scale = p.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int j = 0; j < p.n_tiles; ++j) {
+        int krow, valid;
+        key_tile(p, j, krow, valid);
+        ok = __all_sync(kFull, wait_bounded(&s_full[i], static_cast<uint32_t>(j) & 1u, g, E));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+        tmem_wait_ld();
+        if (valid < 128) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e >= valid) s[c][e] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+        const float mt = mx * scale;
+        if (j == 0) {
+          m_run = mt;
+        } else if (__any_sync(kFull, mt > m_run + 8.f)) {
+          const float m_new = fmaxf(m_run, mt);
+          const float f = ex2_approx(m_run - m_new);
+          l_run *= f;
+          m_run = m_new;
+          ok = __all_sync(kFull,
+                          wait_bounded(&o_done[i], static_cast<uint32_t>(j - 1) & 1u, g, E));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tO + c * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st16(tO + c * 16, o);
+          }
+          tmem_wait_st();
+        }
+        const float neg_m = -m_run;
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = ex2_approx(fmaf(__uint_as_float(s[c][e]), scale, neg_m));
+            const float x1 = ex2_approx(fmaf(__uint_as_float(s[c][e + 1]), scale, neg_m));
+            sum0 += x0;
+            sum1 += x1;
+            const int w = (c * 32 + e) >> 1;  // packed column 0..63
+            pk[w >> 5][w & 31] = pack_bf16x2(x0, x1);
+          }
+        }
+        l_run += sum0 + sum1;
+        tmem_st32(tS, pk[0]);
+        tmem_st32(tS + 32, pk[1]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_ready[i]);
+      }
+      if (ok) {
+        ok = __all_sync(kFull, wait_bounded(&o_done[i],
+                                            static_cast<uint32_t>(p.n_tiles - 1) & 1u, g, E));
+      }
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l_run;
+        const int l = q0 + i * 128 + row;
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
+                             ((static_cast<long long>(b) * p.L + l) * p.H + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          if (l < p.L) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                 __uint_as_float(o[2 * e + 1]) * inv);
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmCols);
+  }
+}
+
+__global__ void wait_timeout_selftest_kernel(int *dev_error, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // nothing ever arrives on it
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitGuard g{&abort_flag, dev_error, limit_ns};
+  const bool ok = __all_sync(kFull, wait_bounded(&bar, 0, g, UNSTEP_ERR_DEVICE_TIMEOUT));
+  if (ok && threadIdx.x == 0) atomicCAS(dev_error, 0, 1);  // impossible: flags a broken wait
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     const AttnParams &p, cudaStream_t stream) {
+  using C = Cfg<D>;
+  // the shared-memory opt-in is per device; remember which devices have it
+  static unsigned long long attr_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (dev >= 64 || !(__atomic_load_n(&attr_set, __ATOMIC_ACQUIRE) & bit)) {
+    e = cudaFuncSetAttribute(window_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
+  }
+  const long long grid = static_cast<long long>(p.B) * p.H * p.n_pairs;
+  if (grid < 1 || grid > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  window_attn_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmemAlloc, stream>>>(
+      tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                               const CUtensorMap &tmap_v, const AttnParams &p,
+                               cudaStream_t stream) {
+  if (D == 128) return launch_d<128>(tmap_q, tmap_k, tmap_v, p, stream);
+  if (D == 64) return launch_d<64>(tmap_q, tmap_k, tmap_v, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(dev_error, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace unstep

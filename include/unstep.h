@@ -1,0 +1,195 @@
+/*
+ * unstep.h -- C ABI of the B200 (sm_100a) chunk-causal attention layer of UnStep's causal video
+ * DiT step.
+ *
+ * Source: "UnStep: Training-Free Acceleration of Causal Video Diffusion with Fewer Steps Than
+ * Distillation" (arXiv 2609.32518).  The abstract names the runtime stack of the DiT: RoPE from
+ * cached coefficients, KV-cache indexing, more efficient attention calls, and a limit on the
+ * temporal window that the attention KV cache retains (Table 1, rows C1 and C4).  Table 3 fixes
+ * the stream: seven causal chunks of three latent frames per 81-frame clip.
+ *
+ * One layer of that step is three operations, exposed as two calls:
+ *   unstep_rope_kv_append  -- 3D RoPE of a chunk's q and k from the cached cos/sin tables,
+ *                             q rotated in place, rotated k and v written into a ring-buffer KV
+ *                             cache that keeps the last cap_frames latent frames (frame f in
+ *                             slot f mod cap_frames);
+ *   unstep_window_attn     -- softmax attention of that chunk's queries over the last `window`
+ *                             latent frames ending at the chunk's last frame (the chunk itself
+ *                             included), scale 1/sqrt(D), fp32 accumulation and softmax.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers into memory the caller allocated and owns.  The
+ *     library never allocates or frees device memory and keeps no pointer beyond a call, except
+ *     the ones the caller stores in unstep_cache_t.
+ *   - Work is enqueued on the caller's stream; no call synchronises the stream, except
+ *     unstep_cache_init (pageable host->device copy of the tables) and unstep_get_device_error.
+ *   - Every call returns UNSTEP_OK (0) or a negative UNSTEP_ERR_* code and never throws.  A call
+ *     that fails on the host leaves the cache and every buffer unchanged.
+ *   - Tensors are bf16, row-major, densely packed.  Activation layout is [B][L][H][D] (stream,
+ *     token, head, channel); token l of a chunk is (i, y, x) with l = i*Hg*Wg + y*Wg + x, i the
+ *     frame inside the chunk.  Cache layout is [B][H][cap_frames*Hg*Wg][D]; frame f's token tok
+ *     lives in row (f mod cap_frames)*Hg*Wg + tok.
+ *   - Pointers must be 16-byte aligned (UNSTEP_ERR_ALIGN otherwise); D must be 64 or 128
+ *     (UNSTEP_ERR_UNSUPPORTED).
+ *   - An unstep_cache_t may not be used from two host threads at once.
+ */
+#ifndef UNSTEP_H_
+#define UNSTEP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st *unstep_stream_t;
+
+enum {
+  UNSTEP_OK = 0,
+  UNSTEP_ERR_ARG = -1,            /* NULL pointer, uninitialised cache, bad scalar */
+  UNSTEP_ERR_SHAPE = -2,          /* shapes disagree with the cache */
+  UNSTEP_ERR_ALIGN = -3,          /* a pointer is not 16-byte aligned */
+  UNSTEP_ERR_FRAME_ORDER = -4,    /* frame_idx is neither the next chunk nor the latest chunk */
+  UNSTEP_ERR_WINDOW = -5,         /* window outside [chunk frames, cap_frames], or empty cache */
+  UNSTEP_ERR_UNSUPPORTED = -6,    /* D not 64/128, or a size beyond the kernels' index range */
+  UNSTEP_ERR_CUDA = -7,           /* a CUDA runtime call failed (launch, copy, memset) */
+  UNSTEP_ERR_DEVICE_TIMEOUT = -8  /* a kernel gave up waiting (reported by the device word) */
+};
+
+/*
+ * One layer's KV cache and RoPE coefficient cache.
+ * The caller fills the shape fields and the five device pointers, then calls unstep_cache_init,
+ * which fills the coefficient tables and the metadata fields.
+ */
+typedef struct {
+  /* shape (caller) */
+  int B;            /* independent streams */
+  int H;            /* heads */
+  int D;            /* head width: 64 or 128 */
+  int Hg, Wg;       /* token grid of one latent frame; T_f = Hg*Wg tokens */
+  int d_t, d_h, d_w;/* RoPE channel blocks, in this order; each even, sum == D */
+  double theta;     /* RoPE base, e.g. 10000 */
+  int cap_frames;   /* ring capacity in latent frames (the retained window W) */
+  int max_pos_t;    /* temporal positions 0 .. max_pos_t-1 are valid frame indices */
+  /* device memory (caller-allocated, caller-owned) */
+  void *k_cache;    /* bf16 [B][H][cap_frames*T_f][D] */
+  void *v_cache;    /* bf16 [B][H][cap_frames*T_f][D] */
+  int *slot_frame;  /* int32 [cap_frames]: frame held by each slot, -1 = empty */
+  float *cos_sin;   /* fp32 coefficient tables, unstep_cache_table_bytes() bytes */
+  int *dev_error;   /* int32 [1]: first device-side error, 0 = none */
+  /* metadata (library-maintained; read-only for the caller) */
+  int frames_written;    /* one past the newest frame written */
+  int first_frame;       /* temporal position of the stream's first frame */
+  int last_chunk_start;  /* first frame of the latest chunk, -1 before any */
+  int last_chunk_frames; /* frames of the latest chunk, 0 before any */
+  int initialized;       /* set by unstep_cache_init */
+} unstep_cache_t;
+
+/* The chunk a call covers: `frames` latent frames of Hg x Wg tokens. */
+typedef struct {
+  int frames, Hg, Wg;
+} unstep_grid_t;
+
+/* Resolved key set of a window: at most two contiguous row ranges of the ring. */
+typedef struct {
+  int first_frame, last_frame; /* frames attended, inclusive */
+  int keys;                    /* (last_frame - first_frame + 1) * T_f */
+  int seg_row[2];              /* first cache row of each range */
+  int seg_len[2];              /* rows in each range; seg_len[1] == 0 when the range is one */
+} unstep_window_plan_t;
+
+/* Library version, e.g. 100 for 0.1.0. */
+int unstep_version(void);
+
+/* Text for a status code (static storage). */
+const char *unstep_status_string(int status);
+
+/* Bytes the caller must allocate for cache->cos_sin (0 if the shape fields are invalid).
+ * Layout: float2 (cos, sin) tables, temporal [max_pos_t][d_t/2], then height [Hg][d_h/2], then
+ * width [Wg][d_w/2]; entry j of position pos holds cos/sin of pos * theta^(-2j/d_a). */
+size_t unstep_cache_table_bytes(const unstep_cache_t *cache);
+
+/* Bytes of ONE of k_cache / v_cache for this shape (0 if invalid). */
+size_t unstep_cache_kv_bytes(const unstep_cache_t *cache);
+
+/*
+ * Validate the shape fields and pointers, compute the coefficient tables on the host in fp64,
+ * round them to fp32 and copy them to cache->cos_sin; zero k_cache, v_cache and dev_error; set
+ * every slot_frame entry to -1; reset the metadata.  Enqueued on `stream`; the table copy is from
+ * pageable memory, so the call returns only after the copy has been staged.
+ * Errors: ARG (NULL pointers, odd or negative split, split sum != D, cap_frames < 1,
+ * max_pos_t < 1, theta <= 0), UNSUPPORTED (D not 64/128, sizes beyond 32-bit row indexing),
+ * ALIGN, CUDA.
+ */
+int unstep_cache_init(unstep_cache_t *cache, unstep_stream_t stream);
+
+/*
+ * Host-only check of an append: the slots frames frame_idx .. frame_idx+grid.frames-1 would
+ * occupy (written to slots_out[0 .. grid.frames-1] if slots_out is non-NULL), and whether the
+ * append is a new chunk (returns 1) or a re-forward of the latest chunk (returns 0).
+ * Rules: grid.Hg/Wg equal the cache's, 1 <= grid.frames <= cap_frames, the frames lie in
+ * [0, max_pos_t); frame_idx is either frames_written (next chunk; any frame_idx >= 0 for the
+ * stream's first chunk) or last_chunk_start with the same frame count (a later denoising step or
+ * the clean-cache pass of the same chunk, which overwrites the same slots).
+ * Errors: ARG, SHAPE, FRAME_ORDER, WINDOW (grid.frames > cap_frames).  Touches no GPU state.
+ */
+int unstep_append_plan(const unstep_cache_t *cache, int frame_idx, unstep_grid_t grid,
+                       int *slots_out);
+
+/*
+ * Fused 3D RoPE + KV-cache append of one chunk (all B streams at the same frame_idx).
+ *   q  : bf16 [B][L][H][D], L = grid.frames*Hg*Wg; rotated IN PLACE.
+ *   k  : bf16 [B][L][H][D], read only; its rotation goes to k_cache.
+ *   v  : bf16 [B][L][H][D], read only; copied bit-exactly to v_cache.
+ * Channel pair (2p, 2p+1) of block a (t, h or w, in that channel order) with in-block index j is
+ * rotated by +ang, ang = pos_a * theta^(-2j/d_a), pos_t = absolute frame index, pos_h = y,
+ * pos_w = x, in fp32 from the fp32 tables, results rounded to bf16 (RNE).  Writes
+ * slot_frame[f mod cap] = f for the chunk's frames and then updates the metadata.
+ * Errors: those of unstep_append_plan, plus ALIGN and CUDA.
+ */
+int unstep_rope_kv_append(void *q, const void *k, const void *v, unstep_cache_t *cache,
+                          int frame_idx, unstep_grid_t grid, unstep_stream_t stream);
+
+/*
+ * Host-only window resolution for the latest chunk: the frames
+ * [max(first_frame, f_end - window + 1), f_end], f_end the latest chunk's last frame, as at
+ * most two contiguous row ranges of the ring.  Errors: ARG, WINDOW (no chunk appended yet, or
+ * window outside [last_chunk_frames, cap_frames]).
+ */
+int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_plan_t *plan);
+
+/*
+ * Windowed chunk-causal attention of the latest chunk.
+ *   q   : bf16 [B][L][H][D], the chunk's ROTATED queries (as unstep_rope_kv_append left them),
+ *         L = last_chunk_frames*Hg*Wg.
+ *   out : bf16 [B][L][H][D]; must not overlap q or the caches.
+ * out = softmax(q K^T / sqrt(D)) V over the window's keys (unstep_window_plan), every query of
+ * the chunk seeing the same keys.  bf16 tensor-core products with fp32 accumulation, fp32
+ * online softmax, output rounded to bf16 (RNE).
+ * Errors: ARG, WINDOW, ALIGN, UNSUPPORTED, CUDA.  A device-side wait that runs past its limit
+ * sets *dev_error (read it with unstep_get_device_error).
+ */
+int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
+                       unstep_stream_t stream);
+
+/*
+ * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported
+ * an error); CUDA if the copy or the synchronisation itself failed.
+ */
+int unstep_get_device_error(const unstep_cache_t *cache, unstep_stream_t stream);
+
+/*
+ * Self-test of the bounded device wait: launches one CTA that waits on a shared-memory barrier
+ * nothing ever completes, giving up after limit_ns nanoseconds; the kernel then writes
+ * UNSTEP_ERR_DEVICE_TIMEOUT to *dev_error (int32 device word) and returns normally, leaving the
+ * context usable.  Errors: ARG, CUDA.
+ */
+int unstep_selftest_wait_timeout(int *dev_error, uint64_t limit_ns, unstep_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UNSTEP_H_ */

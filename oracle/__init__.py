@@ -260,6 +260,23 @@ class OracleLayer:
         self.last_chunk_frames = frames
         return q_rot
 
+    def fill_zero_frames(self, frame_idx: int, frames: int) -> None:
+        """Record a chunk whose rotated keys and values are all zero (no arithmetic: used to
+        bring a cache to a late position quickly when only timing or coverage matters)."""
+        new = self.check_frame_order(frame_idx, frames)
+        for i in range(frames):
+            f = frame_idx + i
+            s = self.slot_of(f)
+            self.K[:, :, s * self.Tf:(s + 1) * self.Tf, :] = 0.0
+            self.V[:, :, s * self.Tf:(s + 1) * self.Tf, :] = 0.0
+            self.slot_frame[s] = f
+        if new:
+            if self.last_chunk_frames == 0:
+                self.first_frame = frame_idx
+            self.frames_written = frame_idx + frames
+        self.last_chunk_start = frame_idx
+        self.last_chunk_frames = frames
+
     def window_frames(self, window: int) -> List[int]:
         """Frames the latest chunk attends to, oldest first."""
         if self.last_chunk_frames == 0:

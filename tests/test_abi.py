@@ -1,0 +1,171 @@
+"""The C ABI without a GPU: the library loads, exports what include/unstep.h declares, and its
+host-side logic (table sizes, frame-order rules, ring slots, window resolution, argument checks)
+agrees with the oracle's.  No call here reaches a kernel launch."""
+import ctypes
+import os
+import random
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from causal_video_diffusion_b200 import binding as B
+from causal_video_diffusion_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "unstep.h")
+INIT_MAGIC = 0x55535450  # the value unstep_cache_init stores in `initialized`
+
+
+@pytest.fixture(scope="module")
+def L():
+    from causal_video_diffusion_b200 import build
+    build.build()
+    return B.lib()
+
+
+def _cache(shape, cap, max_pos_t=128, fake_ptrs=False):
+    c = B.unstep_cache_t()
+    c.B, c.H, c.D, c.Hg, c.Wg = shape.B, shape.H, shape.D, shape.Hg, shape.Wg
+    c.d_t, c.d_h, c.d_w, c.theta = shape.d_t, shape.d_h, shape.d_w, shape.theta
+    c.cap_frames, c.max_pos_t = cap, max_pos_t
+    if fake_ptrs:  # never dereferenced: only calls that fail validation are made with these
+        c.k_cache, c.v_cache, c.slot_frame, c.cos_sin, c.dev_error = (
+            0x100000, 0x200000, 0x300000, 0x400000, 0x500000)
+    return c
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = B.declared_symbols(HEADER)
+    assert set(declared) == set(B._SIGNATURES), declared
+    nm = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                        text=True, check=True).stdout
+    exported = {line.split()[-1] for line in nm.splitlines() if " T " in line}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    for s in declared:
+        assert hasattr(L, s)
+
+
+def test_status_strings(L):
+    for code in range(-8, 1):
+        assert L.unstep_status_string(code)
+    assert L.unstep_status_string(-8) == b"a device-side wait timed out"
+    assert L.unstep_version() == 100
+
+
+def test_table_and_cache_sizes(L):
+    s = W.WORKLOADS["wan_full"].shape
+    c = _cache(s, 21, max_pos_t=120)
+    assert L.unstep_cache_table_bytes(ctypes.byref(c)) == 8 * (120 * 22 + 30 * 21 + 52 * 21)
+    assert L.unstep_cache_kv_bytes(ctypes.byref(c)) == 1 * 12 * 21 * 1560 * 128 * 2
+    c.D, c.d_t = 96, 12        # split still sums to D but D is unsupported
+    assert L.unstep_cache_table_bytes(ctypes.byref(c)) == 0
+    c = _cache(s, 21)
+    c.d_h = 41                 # odd block
+    assert L.unstep_cache_table_bytes(ctypes.byref(c)) == 0
+
+
+def test_init_rejects_bad_arguments_without_touching_the_device(L):
+    s = W.WORKLOADS["tiny"].shape
+    c = _cache(s, 6)
+    assert L.unstep_cache_init(ctypes.byref(c), None) == B.UNSTEP_ERR_ARG      # NULL pointers
+    c = _cache(s, 6, fake_ptrs=True)
+    c.k_cache = 0x100008                                                        # misaligned
+    assert L.unstep_cache_init(ctypes.byref(c), None) == B.UNSTEP_ERR_ALIGN
+    c = _cache(s, 6, fake_ptrs=True)
+    c.theta = -1.0
+    assert L.unstep_cache_init(ctypes.byref(c), None) == B.UNSTEP_ERR_ARG
+    assert L.unstep_cache_init(None, None) == B.UNSTEP_ERR_ARG
+
+
+def _sync_meta(c, ol):
+    c.frames_written = ol.frames_written
+    c.first_frame = ol.first_frame
+    c.last_chunk_start = ol.last_chunk_start
+    c.last_chunk_frames = ol.last_chunk_frames
+    c.initialized = INIT_MAGIC
+
+
+def test_plans_agree_with_the_oracle_ring(L):
+    """Slots, new/re-forward classification and window rows, state by state."""
+    rng = random.Random(3)
+    for trial in range(60):
+        cap = rng.randint(1, 9)
+        frames = rng.randint(1, cap)
+        Hg, Wg = rng.randint(1, 4), rng.randint(1, 5)
+        shape = W.LayerShape(B=1, H=1, D=64, Hg=Hg, Wg=Wg, d_t=24, d_h=20, d_w=20,
+                             chunk_frames=frames)
+        start = rng.choice([0, 0, rng.randint(0, 40)])
+        ol = oracle.OracleLayer(1, 1, Hg, Wg, oracle.RopeSpec(24, 20, 20), cap, heads=[])
+        c = _cache(shape, cap, max_pos_t=400)
+        _sync_meta(c, ol)
+        f = start
+        for step in range(rng.randint(1, 12)):
+            reforward = step > 0 and rng.random() < 0.3
+            fi = ol.last_chunk_start if reforward else f
+            slots = (ctypes.c_int * frames)()
+            rc = L.unstep_append_plan(ctypes.byref(c), fi, B.unstep_grid_t(frames, Hg, Wg), slots)
+            z = np.zeros((1, frames * Hg * Wg, 1, 64), dtype=np.uint16)
+            new = ol.check_frame_order(fi, frames)
+            assert rc == int(new)
+            assert list(slots) == [ol.slot_of(fi + i) for i in range(frames)]
+            ol.append(z, z, z, fi, frames)
+            _sync_meta(c, ol)
+            if not reforward:
+                f += frames
+            for window in range(frames, cap + 1):
+                plan = B.unstep_window_plan_t()
+                assert L.unstep_window_plan(ctypes.byref(c), window, ctypes.byref(plan)) == 0
+                want_frames = ol.window_frames(window)
+                assert (plan.first_frame, plan.last_frame) == (want_frames[0], want_frames[-1])
+                rows = list(range(plan.seg_row[0], plan.seg_row[0] + plan.seg_len[0])) + \
+                    list(range(plan.seg_row[1], plan.seg_row[1] + plan.seg_len[1]))
+                want_rows = [ol.slot_of(fr) * ol.Tf + t for fr in want_frames
+                             for t in range(ol.Tf)]
+                assert rows == want_rows
+                assert plan.keys == len(want_rows)
+
+
+def test_frame_order_and_window_errors(L):
+    s = W.WORKLOADS["tiny"].shape
+    c = _cache(s, 6, fake_ptrs=True)
+    c.initialized = INIT_MAGIC
+    c.frames_written, c.first_frame, c.last_chunk_start, c.last_chunk_frames = 6, 0, 3, 3
+    g = B.unstep_grid_t(3, 4, 6)
+    assert L.unstep_append_plan(ctypes.byref(c), 6, g, None) == 1      # next chunk
+    assert L.unstep_append_plan(ctypes.byref(c), 3, g, None) == 0      # re-forward
+    assert L.unstep_append_plan(ctypes.byref(c), 0, g, None) == B.UNSTEP_ERR_FRAME_ORDER
+    assert L.unstep_append_plan(ctypes.byref(c), 9, g, None) == B.UNSTEP_ERR_FRAME_ORDER
+    assert L.unstep_append_plan(ctypes.byref(c), 3, B.unstep_grid_t(2, 4, 6), None) == \
+        B.UNSTEP_ERR_FRAME_ORDER                                        # re-forward, other size
+    assert L.unstep_append_plan(ctypes.byref(c), 6, B.unstep_grid_t(3, 4, 5), None) == \
+        B.UNSTEP_ERR_SHAPE
+    assert L.unstep_append_plan(ctypes.byref(c), 6, B.unstep_grid_t(7, 4, 6), None) == \
+        B.UNSTEP_ERR_WINDOW                                             # chunk > capacity
+    assert L.unstep_append_plan(ctypes.byref(c), 126, g, None) == B.UNSTEP_ERR_ARG  # > max_pos_t
+    plan = B.unstep_window_plan_t()
+    assert L.unstep_window_plan(ctypes.byref(c), 2, ctypes.byref(plan)) == B.UNSTEP_ERR_WINDOW
+    assert L.unstep_window_plan(ctypes.byref(c), 7, ctypes.byref(plan)) == B.UNSTEP_ERR_WINDOW
+    # the failing calls of the product entry points return before any launch
+    q = ctypes.c_void_p(0x600000)
+    assert L.unstep_rope_kv_append(q, q, q, ctypes.byref(c), 0, g, None) == \
+        B.UNSTEP_ERR_FRAME_ORDER
+    assert L.unstep_rope_kv_append(ctypes.c_void_p(0x600004), q, q, ctypes.byref(c), 6, g,
+                                   None) == B.UNSTEP_ERR_ALIGN
+    assert L.unstep_rope_kv_append(None, q, q, ctypes.byref(c), 6, g, None) == B.UNSTEP_ERR_ARG
+    assert L.unstep_window_attn(q, ctypes.byref(c), 7, q, None) == B.UNSTEP_ERR_WINDOW
+    assert L.unstep_window_attn(ctypes.c_void_p(0x600002), ctypes.byref(c), 6, q, None) == \
+        B.UNSTEP_ERR_ALIGN
+    c2 = _cache(s, 6, fake_ptrs=True)           # never initialised
+    assert L.unstep_window_attn(q, ctypes.byref(c2), 6, q, None) == B.UNSTEP_ERR_ARG
+    # a failed call leaves the metadata unchanged
+    assert (c.frames_written, c.last_chunk_start, c.last_chunk_frames) == (6, 3, 3)
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "_LIB", None)
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="has not been built"):
+        B.lib()

@@ -1,0 +1,250 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (needs a B200).
+
+Small streams whose sizes span several 128-row tiles with ragged tails, ring wrap-around (two key
+segments), re-forwards, streams starting at a later position, B > 1, both head widths; plus the
+closed forms (q = 0 gives the window mean; constant V), determinism, guard regions around every
+buffer, and the bounded-wait self-test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_video_diffusion_b200 import binding
+from causal_video_diffusion_b200 import workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_stream(shape, cap, window, schedule, seed, check_cache=True, heads=None):
+    cache = P.make_cache(shape, cap, max_pos_t=max(f + n for f, n in schedule) + 1)
+    ol = P.make_oracle(shape, cap, heads=heads)
+    hs = ol.heads
+    worst = []
+    for n, (f0, frames) in enumerate(schedule):
+        q, k, v = W.gen_qkv(seed + n, shape)
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        cache.rope_kv_append(qd, kd, vd, f0, frames)
+        out = cache.window_attn(qd, window)
+        torch.cuda.synchronize()
+        assert cache.device_error() == 0
+        q_rot = ol.append(W.bits(q), W.bits(k), W.bits(v), f0, frames)
+        # q rotated in place, within the RoPE rounding bound
+        qg = P.gpu_to_f64(qd)
+        bound = P.rope_error_bound(q_rot, P.gpu_to_f64(q))
+        assert np.all(np.abs(qg - q_rot) <= bound), "rotated q beyond the rounding bound"
+        # k, v were not modified
+        assert torch.equal(kd.cpu(), k) and torch.equal(vd.cpu(), v)
+        if check_cache:
+            P.compare_cache(cache, ol, hs)
+        want = ol.attend(q_rot, window)
+        want = want.reshape(shape.B, len(hs), shape.L, shape.D).transpose(0, 2, 1, 3)
+        got = P.gpu_to_f64(out)[:, :, hs]
+        e = P.attn_errors(got, want)
+        assert e.ok(), (n, f0, e)
+        worst.append(e)
+    return cache, ol, worst
+
+
+def test_tiny_workload():
+    wl = W.WORKLOADS["tiny"]
+    sched = [(wl.frame_idx(c), wl.shape.chunk_frames) for c in range(wl.chunks)]
+    cache, ol, errs = _run_stream(wl.shape, wl.cap, wl.window, sched, seed=1)
+    assert cache.slot_frame.cpu().tolist() == [6, 7, 8, 3, 4, 5]
+    assert max(e.rel_rms for e in errs) < 0.02
+
+
+@pytest.mark.parametrize("D,split", [(64, (24, 20, 20)), (128, (44, 42, 42))])
+@pytest.mark.parametrize("Hg,Wg,frames,cap,window,chunks,start,Bn,H", [
+    (7, 9, 3, 5, 5, 4, 0, 1, 2),      # 189 queries (2 tiles, ragged), wrap of the ring
+    (5, 13, 2, 7, 4, 6, 3, 2, 3),     # window < cap, B = 2, stream starting at frame 3
+    (16, 16, 1, 4, 4, 6, 0, 1, 1),    # 256 queries = exactly two tiles, one-frame chunks
+    (3, 5, 3, 3, 3, 3, 100, 1, 2),    # tiny frames (15 tokens), late positions
+    (11, 23, 3, 9, 9, 3, 0, 1, 2),    # 759 queries: 6 tiles incl. a partial, 1-3 key segments
+])
+def test_streams_match_oracle(D, split, Hg, Wg, frames, cap, window, chunks, start, Bn, H):
+    shape = W.LayerShape(B=Bn, H=H, D=D, Hg=Hg, Wg=Wg, d_t=split[0], d_h=split[1],
+                         d_w=split[2], chunk_frames=frames)
+    sched = []
+    for c in range(chunks):
+        f = start + c * frames
+        sched.append((f, frames))
+        if c == 1:
+            sched.append((f, frames))  # re-forward of the same chunk (next denoising step)
+    _run_stream(shape, cap, window, sched, seed=D + Hg * 7 + cap)
+
+
+def _structured_v(shape, f0):
+    v = torch.zeros(shape.B, shape.L, shape.H, shape.D)
+    l = torch.arange(shape.L)
+    v[..., 0] = 1.0
+    v[..., 1] = (f0 + l // shape.Tf).float()[None, :, None]
+    v[..., 2] = ((l % shape.Tf) % 256).float()[None, :, None] / 256
+    v[..., 3] = -1.0
+    return v.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("D,split,Hg,Wg,cap,window,chunks", [
+    (128, (44, 42, 42), 30, 52, 9, 9, 7),   # the Wan-shaped layer with W = 9, eviction
+    (64, (24, 20, 20), 13, 17, 5, 4, 5),
+])
+def test_zero_query_window_mean(D, split, Hg, Wg, cap, window, chunks):
+    """q = 0 -> all weights equal -> out = mean of V over exactly the window's keys."""
+    shape = W.LayerShape(B=1, H=2, D=D, Hg=Hg, Wg=Wg, d_t=split[0], d_h=split[1], d_w=split[2])
+    cache = P.make_cache(shape, cap, max_pos_t=3 * chunks)
+    for c in range(chunks):
+        f0 = 3 * c
+        _, k, _ = W.gen_qkv(500 + c, shape)
+        q = torch.zeros(shape.B, shape.L, shape.H, shape.D, dtype=torch.bfloat16)
+        v = _structured_v(shape, f0)
+        qd = q.cuda()
+        cache.rope_kv_append(qd, k.cuda(), v.cuda(), f0, 3)
+        out = P.gpu_to_f64(cache.window_attn(qd, window))
+        f_end = f0 + 2
+        frames = list(range(max(0, f_end - window + 1), f_end + 1))
+        exp1 = np.mean(frames)
+        exp2 = np.mean(np.arange(shape.Tf) % 256) / 256
+        for col, val in ((0, 1.0), (1, exp1), (2, exp2), (3, -1.0)):
+            got = out[..., col]
+            tol = P.bf16_ulp(np.array([val]))[0] * 0.51 + 1e-7 * abs(val)
+            assert np.all(np.abs(got - val) <= tol), (c, col, got.min(), got.max(), val)
+        assert np.all(out[..., 4:] == 0)
+
+
+def test_constant_values():
+    shape = W.WORKLOADS["tiny"].shape
+    cache = P.make_cache(shape, 6, max_pos_t=9)
+    v0 = torch.linspace(-3, 3, shape.D).to(torch.bfloat16)
+    for c in range(3):
+        q, k, _ = W.gen_qkv(70 + c, shape)
+        q = q * 4  # peaked softmax: the constant must survive any weighting
+        v = v0.expand(shape.B, shape.L, shape.H, shape.D).contiguous()
+        qd = q.cuda()
+        cache.rope_kv_append(qd, k.cuda(), v.cuda(), 3 * c, 3)
+        out = cache.window_attn(qd, 6).cpu().to(torch.float64)
+        want = v0.to(torch.float64).expand_as(out)
+        assert torch.allclose(out, want, rtol=2 ** -7, atol=1e-6)
+
+
+def test_large_scores_force_rescaling():
+    """Keys whose scores grow chunk after chunk: the running max must be raised correctly."""
+    shape = W.LayerShape(B=1, H=2, D=128, Hg=8, Wg=16, d_t=44, d_h=42, d_w=42)
+    cache = P.make_cache(shape, 6, max_pos_t=18)
+    ol = P.make_oracle(shape, 6)
+    for c in range(6):
+        q, k, v = W.gen_qkv(900 + c, shape)
+        k = (k.float() * (1 + 1.5 * c)).to(torch.bfloat16)     # later keys score much higher
+        q = (q.float() * 2.0).to(torch.bfloat16)
+        qd = q.cuda()
+        cache.rope_kv_append(qd, k.cuda(), v.cuda(), 3 * c, 3)
+        out = P.gpu_to_f64(cache.window_attn(qd, 6))
+        q_rot = ol.append(W.bits(q), W.bits(k), W.bits(v), 3 * c, 3)
+        # scores span tens of units here, so the bf16 rounding of the rotated q and k (which
+        # the cache holds by design) moves them visibly; compare with the oracle's softmax on
+        # those stored values, which isolates the kernel's running-max logic
+        K, V = ol.window_kv(6)
+        Kst = oracle.bf16_to_f64(oracle.f64_to_bf16(K))
+        qst = oracle.bf16_to_f64(oracle.f64_to_bf16(q_rot))
+        rows = [(0, l, h) for h in range(2) for l in range(shape.L)]
+        want = oracle.attention_rows(qst, Kst, V, rows, 1 / np.sqrt(128.0))
+        want = want.reshape(1, 2, shape.L, 128).transpose(0, 2, 1, 3)
+        e = P.attn_errors(out, want)
+        assert e.max_abs < 2e-2 and e.rel_rms < 1e-2, (c, e)
+
+
+def test_deterministic():
+    wl = W.WORKLOADS["tiny"]
+    outs = []
+    for _ in range(2):
+        cache = P.make_cache(wl.shape, wl.cap, max_pos_t=9)
+        o = None
+        for c in range(3):
+            q, k, v = W.gen_qkv(11 + c, wl.shape)
+            qd = q.cuda()
+            cache.rope_kv_append(qd, k.cuda(), v.cuda(), 3 * c, 3)
+            o = cache.window_attn(qd, 6)
+        outs.append((o.cpu(), cache.k_cache.cpu(), cache.v_cache.cpu()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_guard_regions_untouched():
+    """Every buffer sits inside a larger allocation filled with a canary: nothing outside the
+    declared extents may change (a stand-in for a memory checker)."""
+    shape = W.LayerShape(B=2, H=3, D=128, Hg=7, Wg=9, d_t=44, d_h=42, d_w=42)
+    cap, G = 5, 4096  # guard elements on each side
+    L = binding.lib()
+    rows = cap * shape.Tf
+    nkv = shape.B * shape.H * rows * shape.D
+    canary = -12345.0
+
+    def guarded(n, dtype):
+        t = torch.full((n + 2 * G,), canary, dtype=dtype, device="cuda")
+        return t, t[G:G + n]
+
+    kbuf, kc = guarded(nkv, torch.bfloat16)
+    vbuf, vc = guarded(nkv, torch.bfloat16)
+    sbuf, sf = guarded(cap, torch.int32)
+    c = binding.unstep_cache_t()
+    c.B, c.H, c.D, c.Hg, c.Wg = shape.B, shape.H, shape.D, shape.Hg, shape.Wg
+    c.d_t, c.d_h, c.d_w, c.theta, c.cap_frames, c.max_pos_t = 44, 42, 42, 1e4, cap, 30
+    nt = L.unstep_cache_table_bytes(ctypes.byref(c)) // 4
+    tbuf, tab = guarded(nt, torch.float32)
+    ebuf, err = guarded(1, torch.int32)
+    c.k_cache, c.v_cache, c.slot_frame = kc.data_ptr(), vc.data_ptr(), sf.data_ptr()
+    c.cos_sin, c.dev_error = tab.data_ptr(), err.data_ptr()
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.unstep_cache_init(ctypes.byref(c), s) == 0
+    n_act = shape.B * shape.L * shape.H * shape.D
+    bufs = []
+    for c_i in range(4):
+        q, k, v = W.gen_qkv(300 + c_i, shape)
+        qb, qv = guarded(n_act, torch.bfloat16)
+        kb, kv = guarded(n_act, torch.bfloat16)
+        vb, vv = guarded(n_act, torch.bfloat16)
+        ob, ov = guarded(n_act, torch.bfloat16)
+        qv.copy_(q.flatten())
+        kv.copy_(k.flatten())
+        vv.copy_(v.flatten())
+        g = binding.unstep_grid_t(3, shape.Hg, shape.Wg)
+        assert L.unstep_rope_kv_append(qv.data_ptr(), kv.data_ptr(), vv.data_ptr(),
+                                       ctypes.byref(c), 3 * c_i, g, s) == 0
+        assert L.unstep_window_attn(qv.data_ptr(), ctypes.byref(c), 4, ov.data_ptr(), s) == 0
+        bufs += [qb, kb, vb, ob]
+    torch.cuda.synchronize()
+    assert L.unstep_get_device_error(ctypes.byref(c), s) == 0
+    for buf in [kbuf, vbuf, sbuf, tbuf, ebuf] + bufs:
+        head = buf[:G].float()
+        tail = buf[-G:].float()
+        assert torch.all(head == canary) and torch.all(tail == canary)
+
+
+def test_bounded_wait_selftest_reports_timeout_and_context_survives():
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.selftest_wait_timeout(err, limit_ns=2_000_000)      # 2 ms
+    torch.cuda.synchronize()
+    assert int(err.item()) == binding.UNSTEP_ERR_DEVICE_TIMEOUT
+    # the context is still usable: a normal call runs and is correct
+    test_tiny_workload()
+
+
+def test_host_buffer_step_matches_device_path():
+    wl = W.WORKLOADS["tiny"]
+    s = wl.shape
+    a = P.make_cache(s, wl.cap, 9)
+    b = P.make_cache(s, wl.cap, 9)
+    bufs = {n: torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16, device="cuda")
+            for n in ("q", "k", "v", "out")}
+    for c in range(3):
+        q, k, v = W.gen_qkv(40 + c, s)
+        qd = q.cuda()
+        a.rope_kv_append(qd, k.cuda(), v.cuda(), 3 * c, 3)
+        want = a.window_attn(qd, 6).cpu()
+        out_h = torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16).pin_memory()
+        b.step_from_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), 3 * c, 3, 6, out_h,
+                         bufs)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h, want)
