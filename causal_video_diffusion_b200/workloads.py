@@ -106,6 +106,10 @@ WORKLOADS = {
                        forwards_per_chunk=UNSTEP_FORWARDS),
     # 4 independent streams of 120 latent frames (40 chunks), W = 9
     "long_b4": Workload("long_b4", LayerShape(B=4, **WAN), cap=9, window=9, chunks=40),
+    # profiling case: the full-cache layer with 8 of its 12 heads (same kernel, same key count,
+    # inputs still larger than L2, two thirds of the device memory)
+    "wan_full_h8": Workload("wan_full_h8", LayerShape(B=1, **dict(WAN, H=8)), cap=21,
+                            window=21, chunks=7),
 }
 
 

@@ -179,7 +179,7 @@ def test_guard_regions_untouched():
     L = binding.lib()
     rows = cap * shape.Tf
     nkv = shape.B * shape.H * rows * shape.D
-    canary = -12345.0
+    canary = -12288.0  # exact in bf16, fp32 and int32
 
     def guarded(n, dtype):
         t = torch.full((n + 2 * G,), canary, dtype=dtype, device="cuda")
