@@ -71,6 +71,8 @@ _SIGNATURES = {
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),
+    "unstep_selftest_exp2": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                              ctypes.c_void_p], ctypes.c_int),
 }
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -257,6 +259,18 @@ def selftest_wait_timeout(dev_error: torch.Tensor, limit_ns: int,
     _check(lib().unstep_selftest_wait_timeout(_dev_ptr(dev_error, "dev_error"), int(limit_ns),
                                               _stream_handle(stream)),
            "unstep_selftest_wait_timeout")
+
+
+def selftest_exp2(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+    """(polynomial, hardware) base-2 exponentials of the fp32 device tensor x."""
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    yp = torch.empty_like(x)
+    ym = torch.empty_like(x)
+    _check(lib().unstep_selftest_exp2(_dev_ptr(x, "x"), _dev_ptr(yp, "y_poly"),
+                                      _dev_ptr(ym, "y_mufu"), x.numel(), _stream_handle(stream)),
+           "unstep_selftest_exp2")
+    return yp, ym
 
 
 def declared_symbols(header: Optional[str] = None):

@@ -340,4 +340,16 @@ int unstep_selftest_wait_timeout(int *dev_error, uint64_t limit_ns, unstep_strea
   return UNSTEP_OK;
 }
 
+int unstep_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n,
+                         unstep_stream_t stream) {
+  if (!x || !y_poly || !y_mufu || n < 0) return UNSTEP_ERR_ARG;
+  if (n == 0) return UNSTEP_OK;
+  if (unstep::launch_exp2_selftest(x, y_poly, y_mufu, n, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
 }  // extern "C"

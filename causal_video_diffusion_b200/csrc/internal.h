@@ -50,4 +50,7 @@ cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorM
 
 cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cudaStream_t stream);
 
+cudaError_t launch_exp2_selftest(const float *x, float *y_poly, float *y_mufu, int n,
+                                 cudaStream_t stream);
+
 }  // namespace unstep

@@ -126,6 +126,16 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// Per-warpgroup register budgets (all four warps of a warpgroup execute these together).
+template <int N>
+__device__ __forceinline__ void regs_release() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_claim() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -149,6 +159,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
   return d;
+}
+
+// A 64-bit descriptor from its 32-bit halves.
+__device__ __forceinline__ uint64_t f2u64(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
 }
 
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32 accumulator:
@@ -256,6 +273,68 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed pairs of fp32 values (low, high) for the sm_100 f32x2 arithmetic.
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe instead of MUFU.  Range reduction splits
+// x = n + f exactly, n = round-to-nearest(x) obtained by adding and subtracting 1.5 * 2^23
+// (fp32 round-to-nearest), f in [-1/2, 1/2]; 2^f is a degree-3 polynomial whose coefficients are
+// the minimax (Remez exchange) fit of the relative error on [-1/2, 1/2] (max relative error
+// 7.5e-5, below bf16's half-ulp 2^-9; see exp2_poly_remez.py beside this file); 2^n is applied by
+// adding n to the exponent field.  Valid for x in [-125, 127]: callers clamp from below, and
+// x <= 8 here because the running max is never more than 8 below a tile's scores.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t x = f2_make(x0, x1);
+  const uint64_t magic = f2_make(12582912.f, 12582912.f);
+  const uint64_t neg_magic = f2_make(-12582912.f, -12582912.f);
+  const uint64_t minus1 = f2_make(-1.f, -1.f);
+  const uint64_t t = fadd2(x, magic);         // n in the low mantissa bits
+  const uint64_t n = fadd2(t, neg_magic);     // n as a float
+  const uint64_t f = ffma2(n, minus1, x);     // x - n, exact
+  uint64_t p = ffma2(f2_make(kExp2C3, kExp2C3), f, f2_make(kExp2C2, kExp2C2));
+  p = ffma2(p, f, f2_make(kExp2C1, kExp2C1));
+  p = ffma2(p, f, f2_make(kExp2C0, kExp2C0));
+  float t0, t1, p0, p1;
+  f2_split(t, t0, t1);
+  f2_split(p, p0, p1);
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2_make(r0, r1);
 }
 
 // Two floats -> packed bf16x2 (RNE); `lo` lands in the low 16 bits.

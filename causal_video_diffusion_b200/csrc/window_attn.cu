@@ -10,12 +10,13 @@
 //   O   += P_j V_j                      tcgen05.mma, A = P_j (TMEM, aliasing S_j), B = V_j (smem)
 //   l   += rowsum(P_j);   out = O / l  (bf16)
 //
-// Work split of one CTA (one (stream, head) and two 128-row query tiles, 320 threads):
+// Work split of one CTA (one (stream, head) and two 128-row query tiles, 384 threads):
 //   warps 0-3  softmax + epilogue of query tile 0 (thread t owns TMEM lane / query row t)
 //   warps 4-7  softmax + epilogue of query tile 1
 //   warp  8    TMA producer: Q once, then K_0, V_0, K_1, V_1, ... through an NS-stage ring
 //   warp  9    MMA issuer (one thread): QK^T and PV for both tiles, ping-ponging so that the
 //              tensor core works on one tile while the other tile's softmax runs
+//   warps 10-11 idle (they complete the third warpgroup, whose registers the softmax takes)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 //
 // The ring cache holds the window as at most two contiguous row ranges; each range is tiled on
@@ -35,7 +36,20 @@
 namespace unstep {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Register split: launched at 168 per thread (384 x 168 = 64512), the producer/MMA warpgroup
+// drops to kRegsIo and the two softmax warpgroups rise to kRegsSoftmax; the static_assert keeps
+// 2 x 128 x kRegsSoftmax + 128 x kRegsIo within the launch total (208/80: 63488), so the claim
+// can always be satisfied.
+#ifndef UNSTEP_REGS_SOFTMAX
+#define UNSTEP_REGS_SOFTMAX 208
+#endif
+#ifndef UNSTEP_REGS_IO
+#define UNSTEP_REGS_IO 80
+#endif
+constexpr int kRegsSoftmax = UNSTEP_REGS_SOFTMAX;
+constexpr int kRegsIo = UNSTEP_REGS_IO;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * 168, "register split");
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
@@ -73,6 +87,65 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > kDrainLimitNs) return;
   }
+}
+
+// Share of the exponentials computed on the FMA pipe (exp2_poly2) instead of MUFU: in every 8
+// column pairs of a 128-key tile, the last kEmuPairsPer8 pairs.  MUFU alone (16 per clock per SM)
+// needs as long for one tile's 16384 exponentials as the tensor core needs for the other tile's
+// two 128x128x128 products, so moving part of them to the FMA pipe shortens the softmax phase.
+#ifndef UNSTEP_EMU_PAIRS_PER8
+#define UNSTEP_EMU_PAIRS_PER8 3
+#endif
+constexpr int kEmuPairsPer8 = UNSTEP_EMU_PAIRS_PER8;
+
+// Max of a row's 128 scores: eight independent chains of 3-input max, then a short tree.
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
+  float m8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = k >> 1, e0 = (k & 1) * 16;
+    float m = fmax3(__uint_as_float(s[c][e0]), __uint_as_float(s[c][e0 + 1]),
+                    __uint_as_float(s[c][e0 + 2]));
+#pragma unroll
+    for (int e = 3; e < 15; e += 2)
+      m = fmax3(m, __uint_as_float(s[c][e0 + e]), __uint_as_float(s[c][e0 + e + 1]));
+    m8[k] = fmaxf(m, __uint_as_float(s[c][e0 + 15]));
+  }
+  return fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+}
+
+// P for one 32-column chunk of a row: p = 2^(s * scale - m), summed into acc (four packed
+// accumulators), rounded to bf16 pairs and stored to the 16 TMEM columns at `taddr` (the P
+// columns alias the S columns already read).  kMasked: columns >= valid are zero (a segment's
+// last, partial tile), all exponentials on MUFU so that masked ones are exactly 0.
+template <bool kMasked>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], int col0, int valid,
+                                          uint64_t sc2, uint64_t nm2, uint64_t (&acc)[4],
+                                          uint32_t taddr) {
+  uint32_t w[16];
+#pragma unroll
+  for (int pi = 0; pi < 16; ++pi) {
+    const uint64_t x2 = ffma2(f2_make(__uint_as_float(s[2 * pi]), __uint_as_float(s[2 * pi + 1])),
+                              sc2, nm2);
+    uint64_t p2;
+    if (!kMasked && (pi & 7) >= 8 - kEmuPairsPer8) {
+      p2 = exp2_poly2(x2);
+    } else {
+      float x0, x1;
+      f2_split(x2, x0, x1);
+      float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      if (kMasked) {
+        p0 = (col0 + 2 * pi < valid) ? p0 : 0.f;
+        p1 = (col0 + 2 * pi + 1 < valid) ? p1 : 0.f;
+      }
+      p2 = f2_make(p0, p1);
+    }
+    acc[pi & 3] = fadd2(acc[pi & 3], p2);
+    float p0, p1;
+    f2_split(p2, p0, p1);
+    w[pi] = pack_bf16x2(p0, p1);
+  }
+  tmem_st16(taddr, w);
 }
 
 template <int D>
@@ -131,6 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitGuard g{abort_flag, p.dev_error, p.wait_limit_ns};
   constexpr int E = UNSTEP_ERR_DEVICE_TIMEOUT;
 
+  if (warp >= 8) {
+    regs_release<kRegsIo>();
   if (warp == 8) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -173,24 +248,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
       const uint32_t sQ = smem_u32(smem + C::kSmemQ);
       const uint32_t sKV = smem_u32(smem + C::kSmemKV);
+      // descriptors as 32-bit halves: the high half (stride offset, version, swizzle) is the
+      // same for every operand of a kind; only the start address in the low half moves
+      const uint32_t kHiK = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
+      const uint32_t kHiV = static_cast<uint32_t>(sdesc_sw128(0, 16384, 1024) >> 32);
+      const uint32_t loQ = static_cast<uint32_t>(sdesc_sw128(sQ, 16, 1024));
+      const uint32_t loK = static_cast<uint32_t>(sdesc_sw128(sKV, 16, 1024));
+      const uint32_t loV = static_cast<uint32_t>(sdesc_sw128(sKV, 16384, 1024));
       auto qk = [&](int t, int s) {
         const uint32_t dS = tmem + (t ? C::kTmS1 : C::kTmS0);
+        const uint32_t qa = loQ + static_cast<uint32_t>(t * (C::kTileBytes >> 4));
+        const uint32_t kb = loK + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
-          const uint64_t a = sdesc_sw128(sQ + t * C::kTileBytes + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKV + s * C::kTileBytes + off, 16, 1024);
-          umma_ss(dS, a, bd, kIdQK, kk > 0 ? 1u : 0u);
+          const uint32_t off = static_cast<uint32_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          umma_ss(dS, f2u64(qa + off, kHiK), f2u64(kb + off, kHiK), kIdQK, kk > 0 ? 1u : 0u);
         }
       };
       auto pv = [&](int t, int s, bool acc) {
         const uint32_t dO = tmem + (t ? C::kTmO1 : C::kTmO0);
         const uint32_t aP = tmem + (t ? C::kTmS1 : C::kTmS0);
+        const uint32_t vb = loV + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = sdesc_sw128(sKV + s * C::kTileBytes + kk * 2048, 16384, 1024);
-          umma_ts(dO, aP + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(dO, aP + kk * 8, f2u64(vb + static_cast<uint32_t>(kk * (2048 >> 4)), kHiV),
+                  kIdPV, (acc || kk > 0) ? 1u : 0u);
       };
       auto wait_full = [&](int n) {
         return wait_bounded(&full[n % NS], static_cast<uint32_t>(n / NS) & 1u, g, E);
@@ -242,7 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(drain, 0);
     }
     __syncwarp();
+  }
   } else {
+    regs_claim<kRegsSoftmax>();
     // ---------------------------------------------------------------- softmax + epilogue
     const int i = warp >> 2;          // query tile of this warpgroup
     const int wq = warp & 3;          // TMEM lane quarter
@@ -264,19 +348,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
         tmem_wait_ld();
-        if (valid < 128) {
+        const bool masked = valid < 128;
+        if (masked) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
               if (c * 32 + e >= valid) s[c][e] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
-        const float mt = mx * scale;
+        const float mt = row_max128(s) * scale;
         if (j == 0) {
           m_run = mt;
         } else if (__any_sync(kFull, mt > m_run + 8.f)) {
@@ -299,24 +379,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
         }
-        const float neg_m = -m_run;
-        float sum0 = 0.f, sum1 = 0.f;
-        uint32_t pk[2][32];
+        const uint64_t sc2 = f2_make(scale, scale);
+        const uint64_t nm2 = f2_make(-m_run, -m_run);
+        uint64_t acc[4] = {0, 0, 0, 0};
+        if (!masked) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 4; ++c) exp_chunk<false>(s[c], c * 32, 128, sc2, nm2, acc, tS + c * 16);
+        } else {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float x0 = ex2_approx(fmaf(__uint_as_float(s[c][e]), scale, neg_m));
-            const float x1 = ex2_approx(fmaf(__uint_as_float(s[c][e + 1]), scale, neg_m));
-            sum0 += x0;
-            sum1 += x1;
-            const int w = (c * 32 + e) >> 1;  // packed column 0..63
-            pk[w >> 5][w & 31] = pack_bf16x2(x0, x1);
-          }
+          for (int c = 0; c < 4; ++c) exp_chunk<true>(s[c], c * 32, valid, sc2, nm2, acc, tS + c * 16);
         }
-        l_run += sum0 + sum1;
-        tmem_st32(tS, pk[0]);
-        tmem_st32(tS + 32, pk[1]);
+        {
+          float a0, a1, b0, b1;
+          f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+          (void)b0;
+          (void)b1;
+          l_run += a0 + a1;
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_ready[i]);
@@ -374,6 +453,21 @@ __global__ void wait_timeout_selftest_kernel(int *dev_error, uint64_t limit_ns) 
   if (ok && threadIdx.x == 0) atomicCAS(dev_error, 0, 1);  // impossible: flags a broken wait
 }
 
+__global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_mufu, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = 2 * i;
+  if (j >= n) return;
+  const float x0 = x[j], x1 = (j + 1 < n) ? x[j + 1] : 0.f;
+  float p0, p1;
+  f2_split(exp2_poly2(f2_make(x0, x1)), p0, p1);
+  y_poly[j] = p0;
+  y_mufu[j] = ex2_approx(x0);
+  if (j + 1 < n) {
+    y_poly[j + 1] = p1;
+    y_mufu[j + 1] = ex2_approx(x1);
+  }
+}
+
 template <int D>
 cudaError_t launch_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      const AttnParams &p, cudaStream_t stream) {
@@ -405,6 +499,13 @@ cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorM
   if (D == 128) return launch_d<128>(tmap_q, tmap_k, tmap_v, p, stream);
   if (D == 64) return launch_d<64>(tmap_q, tmap_k, tmap_v, p, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_exp2_selftest(const float *x, float *y_poly, float *y_mufu, int n,
+                                 cudaStream_t stream) {
+  const int pairs = (n + 1) / 2;
+  exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y_poly, y_mufu, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cudaStream_t stream) {

@@ -188,6 +188,16 @@ int unstep_get_device_error(const unstep_cache_t *cache, unstep_stream_t stream)
  */
 int unstep_selftest_wait_timeout(int *dev_error, uint64_t limit_ns, unstep_stream_t stream);
 
+/*
+ * Self-test of the attention kernel's two base-2 exponentials on n device floats x (fp32):
+ * y_poly[i] = the FMA-pipe polynomial (exact range split x = n + f, degree-3 minimax fit of
+ * 2^f on [-1/2, 1/2]; inputs below -125 are clamped to -125), y_mufu[i] = the hardware ex2.approx.
+ * No counterpart in the paper: it lets a test bound the polynomial's error against both CUDA's
+ * instruction and the exact value.  Errors: ARG, CUDA.
+ */
+int unstep_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int n,
+                         unstep_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -169,3 +169,19 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="has not been built"):
         B.lib()
+
+
+def test_exp2_polynomial_coefficients_match_their_derivation():
+    """The constants in the kernel header are the Remez fit the derivation script produces."""
+    import re
+    import importlib.util
+    root = ROOT
+    hdr = open(os.path.join(root, "causal_video_diffusion_b200", "csrc", "sm100.cuh")).read()
+    consts = [float(v) for v in re.findall(r"kExp2C\d = ([0-9.eE+-]+)f;", hdr)]
+    spec = importlib.util.spec_from_file_location(
+        "remez", os.path.join(root, "causal_video_diffusion_b200", "csrc", "exp2_poly_remez.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    c = np.float32(m.remez_exp2())
+    assert np.allclose(consts, c, rtol=0, atol=1e-7)
+    assert m.max_rel_err(c) < 8e-5

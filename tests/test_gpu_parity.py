@@ -248,3 +248,21 @@ def test_host_buffer_step_matches_device_path():
                          bufs)
         torch.cuda.synchronize()
         assert torch.equal(out_h, want)
+
+
+def test_exp2_polynomial_against_hardware_and_exact():
+    """The FMA-pipe 2^x matches the exact value to 1e-4 relative over the whole range the
+    softmax feeds it, and agrees with the hardware ex2 to the same bound."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001),
+                   torch.tensor([-0.5, 0.5, 0.0, -1e-7, 1e-7, -124.99, 7.9999])]).cuda()
+    yp, ym = binding.selftest_exp2(x)
+    xd = x.double().cpu()
+    exact = torch.exp2(xd)
+    rel_p = ((yp.double().cpu() - exact).abs() / exact).max().item()
+    rel_m = ((ym.double().cpu() - exact).abs() / exact).max().item()
+    assert rel_p < 1e-4, rel_p
+    assert rel_m < 1e-5, rel_m
+    assert (((yp - ym).abs() / ym).max().item()) < 1.1e-4
+    # below the clamp the polynomial returns 2^-125, never a negative or NaN value
+    y_low, _ = binding.selftest_exp2(torch.tensor([-200.0, -1e30], device="cuda"))
+    assert torch.all(y_low == torch.tensor(2.0 ** -125, device="cuda"))

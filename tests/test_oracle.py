@@ -363,3 +363,4 @@ def test_clip_schedule_matches_table3():
     assert all(n == g["unstep_steps_later"][0] + clean for n in W.UNSTEP_FORWARDS[1:])
     # 60x104 latent, 2x2 patches -> 30x52 tokens per latent frame
     assert (wl.shape.Hg * 2, wl.shape.Wg * 2) == tuple(g["noise_shape"][3:5])
+
