@@ -36,6 +36,7 @@ class unstep_cache_t(ctypes.Structure):
         ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
         ("slot_frame", ctypes.c_void_p), ("cos_sin", ctypes.c_void_p),
         ("dev_error", ctypes.c_void_p),
+        ("attn_scratch", ctypes.c_void_p), ("attn_scratch_bytes", ctypes.c_size_t),
         ("frames_written", ctypes.c_int), ("first_frame", ctypes.c_int),
         ("last_chunk_start", ctypes.c_int), ("last_chunk_frames", ctypes.c_int),
         ("initialized", ctypes.c_int),
@@ -58,6 +59,7 @@ _SIGNATURES = {
     "unstep_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "unstep_cache_table_bytes": ([ctypes.POINTER(unstep_cache_t)], ctypes.c_size_t),
     "unstep_cache_kv_bytes": ([ctypes.POINTER(unstep_cache_t)], ctypes.c_size_t),
+    "unstep_attn_scratch_bytes": ([ctypes.POINTER(unstep_cache_t)], ctypes.c_size_t),
     "unstep_cache_init": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_append_plan": ([ctypes.POINTER(unstep_cache_t), ctypes.c_int, unstep_grid_t,
                             ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -136,7 +138,8 @@ class LayerCache:
     def __init__(self, B: int, H: int, D: int, Hg: int, Wg: int, d_t: int, d_h: int, d_w: int,
                  cap_frames: int, max_pos_t: int, theta: float = 10000.0,
                  device: Optional[torch.device] = None,
-                 stream: Optional[torch.cuda.Stream] = None):
+                 stream: Optional[torch.cuda.Stream] = None,
+                 scratch: Optional[torch.Tensor] = None, use_scratch: bool = True):
         L = lib()
         dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                            torch.cuda.current_device())
@@ -159,6 +162,21 @@ class LayerCache:
         c.slot_frame = self.slot_frame.data_ptr()
         c.cos_sin = self.cos_sin.data_ptr()
         c.dev_error = self.dev_error.data_ptr()
+        # attention scratch: given (shared between caches on one stream), or allocated here
+        self.scratch = None
+        if use_scratch:
+            with torch.cuda.device(dev):
+                need = L.unstep_attn_scratch_bytes(ctypes.byref(c))
+            if need == 0:
+                raise UnstepError(UNSTEP_ERR_ARG, "attention scratch size")
+            if scratch is None:
+                scratch = torch.empty((need,), dtype=torch.uint8, device=dev)
+            if scratch.numel() * scratch.element_size() < need:
+                raise ValueError(f"scratch has {scratch.numel() * scratch.element_size()} bytes, "
+                                 f"needs {need}")
+            self.scratch = scratch
+            c.attn_scratch = scratch.data_ptr()
+            c.attn_scratch_bytes = scratch.numel() * scratch.element_size()
         self.c = c
         self.device = dev
         with torch.cuda.device(dev):

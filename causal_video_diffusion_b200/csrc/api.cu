@@ -3,6 +3,7 @@
 //
 // UnStep paper (arXiv 2609.32518), abstract: RoPE "with cached coefficients", KV indexing and a
 // limited temporal window of the attention KV cache; Table 3: chunks of three latent frames.
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -85,6 +86,42 @@ bool encode_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *d
   return r == CUDA_SUCCESS;
 }
 
+// Multiprocessor count of the current device (cached per device).
+int device_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0 && dev < 64) {
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+long long max_units(const unstep_cache_t *c) {
+  const long long rows = static_cast<long long>(c->cap_frames) * c->Hg * c->Wg;
+  return static_cast<long long>(c->B) * c->H * ((rows + 255) / 256);
+}
+
+size_t scratch_bytes_for(const unstep_cache_t *c, int sms) {
+  return unstep::attn_counter_bytes(max_units(c)) +
+         2ull * static_cast<size_t>(sms) * unstep::attn_slot_floats(c->D) * sizeof(float);
+}
+
+unsigned next_epoch() {
+  static std::atomic<unsigned> counter{0};
+  return counter.fetch_add(1, std::memory_order_relaxed) % 0xFFFFFFu + 1u;
+}
+
 }  // namespace
 
 extern "C" {
@@ -117,14 +154,27 @@ size_t unstep_cache_kv_bytes(const unstep_cache_t *cache) {
          cache->D * 2;
 }
 
+size_t unstep_attn_scratch_bytes(const unstep_cache_t *cache) {
+  if (check_shape(cache)) return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  return scratch_bytes_for(cache, sms);
+}
+
 int unstep_cache_init(unstep_cache_t *cache, unstep_stream_t stream) {
   int rc = check_shape(cache);
   if (rc) return rc;
   if (!cache->k_cache || !cache->v_cache || !cache->slot_frame || !cache->cos_sin ||
       !cache->dev_error)
     return UNSTEP_ERR_ARG;
-  if (!aligned16(cache->k_cache) || !aligned16(cache->v_cache) || !aligned16(cache->cos_sin))
+  if (!aligned16(cache->k_cache) || !aligned16(cache->v_cache) || !aligned16(cache->cos_sin) ||
+      !aligned16(cache->attn_scratch))
     return UNSTEP_ERR_ALIGN;
+  if (cache->attn_scratch) {
+    const int sms = device_sms();
+    if (sms <= 0) return UNSTEP_ERR_CUDA;
+    if (cache->attn_scratch_bytes < scratch_bytes_for(cache, sms)) return UNSTEP_ERR_ARG;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // cached coefficients: cos/sin of pos * theta^(-2j/d_a), computed in fp64, stored fp32
   std::vector<float> tab(table_floats(cache));
@@ -149,7 +199,10 @@ int unstep_cache_init(unstep_cache_t *cache, unstep_stream_t stream) {
       cudaMemsetAsync(cache->v_cache, 0, kvb, s) != cudaSuccess ||
       cudaMemsetAsync(cache->slot_frame, 0xFF, sizeof(int) * cache->cap_frames, s) !=
           cudaSuccess ||
-      cudaMemsetAsync(cache->dev_error, 0, sizeof(int), s) != cudaSuccess) {
+      cudaMemsetAsync(cache->dev_error, 0, sizeof(int), s) != cudaSuccess ||
+      (cache->attn_scratch &&
+       cudaMemsetAsync(cache->attn_scratch, 0, unstep::attn_counter_bytes(max_units(cache)), s) !=
+           cudaSuccess)) {
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
   }
@@ -300,12 +353,41 @@ int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, v
   p.H = H;
   p.L = L;
   p.n_pairs = (L + 255) / 256;
+  p.n_units = B * H * p.n_pairs;
   for (int s = 0; s < 2; ++s) {
     p.seg_row[s] = plan.seg_row[s];
     p.seg_len[s] = plan.seg_len[s];
     p.seg_tiles[s] = (plan.seg_len[s] + 127) / 128;
   }
   p.n_tiles = p.seg_tiles[0] + p.seg_tiles[1];
+  p.div_pairs = unstep::make_fastdiv(static_cast<uint32_t>(p.n_pairs));
+  p.div_heads = unstep::make_fastdiv(static_cast<uint32_t>(H));
+  // persistent schedule: whole units in waves of `sms` CTAs, the remainder split along keys
+  const int sms = cache->attn_scratch ? device_sms() : 0;
+  if (cache->attn_scratch && sms > 0) {
+    const int U = p.n_units;
+    p.dp_waves = U / sms;
+    const int tail = U - p.dp_waves * sms;
+    p.u_tail0 = p.dp_waves * sms;
+    p.w_tail = static_cast<long long>(tail) * p.n_tiles;
+    long long gsk = tail > 0 ? static_cast<long long>(tail) * 8 : 0;  // at most ~8 pieces/unit
+    if (gsk > sms) gsk = sms;
+    if (gsk > p.w_tail) gsk = p.w_tail;
+    p.g_sk = static_cast<int>(gsk);
+    p.grid = p.dp_waves > 0 ? sms : p.g_sk;
+    p.counters = static_cast<unsigned *>(cache->attn_scratch);
+    p.slots = reinterpret_cast<float *>(static_cast<char *>(cache->attn_scratch) +
+                                        unstep::attn_counter_bytes(max_units(cache)));
+    p.slot_floats = static_cast<int>(unstep::attn_slot_floats(D));
+    p.epoch = next_epoch();
+  } else {
+    // no scratch: one CTA per unit, nothing is split
+    p.dp_waves = 1;
+    p.grid = p.n_units;
+    p.u_tail0 = p.n_units;
+    p.g_sk = 0;
+    p.w_tail = 0;
+  }
   p.scale_log2 = static_cast<float>(1.4426950408889634073599 / std::sqrt(static_cast<double>(D)));
   p.wait_limit_ns = unstep::kWaitLimitNs;
   if (unstep::launch_window_attn(D, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) !=

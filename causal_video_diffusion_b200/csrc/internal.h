@@ -29,18 +29,60 @@ struct RopeAppendParams {
 
 cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream);
 
+// Division by a run-time invariant d by multiply-high (Granlund & Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, x / d = (umulhi(x, m) + x) >> l for 0 <= x < 2^31.
+struct FastDiv {
+  uint32_t d, m, l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  const uint64_t m = ((1ull << 32) * ((1ull << l) - d)) / d + 1;
+  return FastDiv{d, static_cast<uint32_t>(m), l};
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv &f) {
+  return (__umulhi(x, f.m) + x) >> f.l;
+}
+#endif
+
 struct AttnParams {
   void *out;         // bf16 [B][L][H][D]
   int *dev_error;
   int B, H, L;
-  int n_pairs;       // CTAs per (b, h): two 128-row query tiles each
+  int n_pairs;       // units per (b, h): two 128-row query tiles each
+  int n_units;       // B * H * n_pairs
   int n_tiles;       // key tiles of 128 rows over both ring segments
   int seg_row[2];
   int seg_len[2];
   int seg_tiles[2];
   float scale_log2;  // log2(e) / sqrt(D)
   uint64_t wait_limit_ns;
+  // persistent schedule: dp_waves whole units per CTA, then the tail units
+  // [u_tail0, n_units) cut into w_tail = (n_units - u_tail0) * n_tiles key tiles over g_sk CTAs
+  int grid;
+  int dp_waves;
+  int u_tail0;
+  int g_sk;
+  long long w_tail;
+  // scratch of split units: per-(unit, query tile) counts and two slots per CTA of
+  // slot_floats floats each (per query tile: O[D][128], m[128], l[128])
+  unsigned *counters;
+  float *slots;
+  int slot_floats;
+  unsigned epoch;    // 1 .. 2^24-1, distinct for consecutive launches
+  FastDiv div_pairs; // by n_pairs
+  FastDiv div_heads; // by H
 };
+
+// Scratch layout shared by the host sizing and the kernel.
+constexpr size_t attn_counter_bytes(long long max_units) {
+  return ((static_cast<size_t>(max_units) * 2 * sizeof(unsigned) + 255) / 256) * 256;
+}
+constexpr size_t attn_slot_floats(int D) { return 2 * (static_cast<size_t>(D) * 128 + 256); }
 
 // tmap_q: 4D (D, H, L, B) bf16, box (64, 1, 128, 1), 128B swizzle.
 // tmap_k / tmap_v: 3D (D, cap*T_f, B*H) bf16, box (64, 128, 1), 128B swizzle.

@@ -39,13 +39,13 @@ namespace {
 constexpr int kThreads = 384;
 // Register split: launched at 168 per thread (384 x 168 = 64512), the producer/MMA warpgroup
 // drops to kRegsIo and the two softmax warpgroups rise to kRegsSoftmax; the static_assert keeps
-// 2 x 128 x kRegsSoftmax + 128 x kRegsIo within the launch total (208/80: 63488), so the claim
+// 2 x 128 x kRegsSoftmax + 128 x kRegsIo within the launch total (200/96: 63488), so the claim
 // can always be satisfied.
 #ifndef UNSTEP_REGS_SOFTMAX
-#define UNSTEP_REGS_SOFTMAX 208
+#define UNSTEP_REGS_SOFTMAX 200
 #endif
 #ifndef UNSTEP_REGS_IO
-#define UNSTEP_REGS_IO 80
+#define UNSTEP_REGS_IO 96
 #endif
 constexpr int kRegsSoftmax = UNSTEP_REGS_SOFTMAX;
 constexpr int kRegsIo = UNSTEP_REGS_IO;
@@ -148,6 +148,182 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], int col0, int
   tmem_st16(taddr, w);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Work decomposition.  A unit is one (stream, head) with two 128-row query tiles over all of the
+// window's key tiles; units are numbered head-major, u = (b*H + h)*n_pairs + pair.  The grid is
+// persistent: CTA c first takes whole units in dp_waves data-parallel waves (unit w*grid + c, so
+// that concurrent CTAs share a head's K/V in L2), then its share of the remaining tail units'
+// key tiles, cut evenly over g_sk CTAs (stream-K).  A tail unit split between CTAs leaves each
+// piece's unnormalised O, running max and row sum in a scratch slot; the last CTA to finish a
+// piece of it (an atomic count per unit and query tile) merges them.  No CTA waits for another.
+// ---------------------------------------------------------------------------------------------
+struct Seg {
+  int u;        // unit
+  int k0, k1;   // key tiles [k0, k1) of the unit
+  int slot;     // scratch slot of a partial segment (2c or 2c+1), -1 when the unit is whole
+};
+
+__device__ __forceinline__ long long sk_lo(const AttnParams &p, int c) {
+  return static_cast<long long>(c) * p.w_tail / p.g_sk;
+}
+
+// This CTA's share [lo, hi) of the tail's key tiles, computed once.
+struct SkRange {
+  long long lo, hi;
+  long long u_rel0;  // tail unit holding tile lo
+};
+
+__device__ __forceinline__ SkRange sk_range(const AttnParams &p, int c) {
+  SkRange r{0, 0, 0};
+  if (c < p.g_sk) {
+    r.lo = sk_lo(p, c);
+    r.hi = sk_lo(p, c + 1);
+    r.u_rel0 = r.lo / p.n_tiles;
+  }
+  return r;
+}
+
+// The q-th segment of CTA c; false when the CTA has no more.
+__device__ __forceinline__ bool get_seg(const AttnParams &p, int c, const SkRange &sk, int q,
+                                        Seg &s) {
+  if (q < p.dp_waves) {
+    s.u = q * p.grid + c;
+    s.k0 = 0;
+    s.k1 = p.n_tiles;
+    s.slot = -1;
+    return true;
+  }
+  const int r = q - p.dp_waves;
+  if (c >= p.g_sk || r > 1) return false;
+  const long long u_rel = sk.u_rel0 + r;
+  const long long us = u_rel * p.n_tiles;
+  if (us >= sk.hi) return false;
+  s.u = p.u_tail0 + static_cast<int>(u_rel);
+  s.k0 = static_cast<int>((sk.lo > us ? sk.lo : us) - us);
+  s.k1 = static_cast<int>((sk.hi < us + p.n_tiles ? sk.hi : us + p.n_tiles) - us);
+  s.slot = (s.k0 == 0 && s.k1 == p.n_tiles) ? -1 : 2 * c + r;
+  return true;
+}
+
+struct UnitPos {
+  int b, h, bh, q0;
+  bool has1;
+};
+
+__device__ __forceinline__ UnitPos unit_pos(const AttnParams &p, int u) {
+  UnitPos x;
+  x.bh = static_cast<int>(fdiv(static_cast<uint32_t>(u), p.div_pairs));
+  const int pair = u - x.bh * p.n_pairs;
+  x.b = static_cast<int>(fdiv(static_cast<uint32_t>(x.bh), p.div_heads));
+  x.h = x.bh - x.b * p.H;
+  x.q0 = pair * 256;
+  x.has1 = x.q0 + 128 < p.L;
+  return x;
+}
+
+// Named barrier of one softmax warpgroup (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void wg_sync(int i) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + i) : "memory");
+}
+
+// Cold per-segment work of a softmax thread (one query row).  Inlined by default (measured
+// faster on B200 than out-of-line calls, whose register saves cost more than they free);
+// UNSTEP_COLD_NOINLINE moves them out of line.
+#ifdef UNSTEP_COLD_NOINLINE
+#define UNSTEP_COLD_FN __device__ __noinline__
+#else
+#define UNSTEP_COLD_FN __device__ __forceinline__
+#endif
+
+// O row / l -> bf16, stored to dst (the row's D channels) when `live` (row < L).
+template <int D>
+UNSTEP_COLD_FN void store_row(uint32_t tO, float inv, __nv_bfloat16 *dst, bool live) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(tO + c * 32, o);
+    tmem_wait_ld();
+    if (live) {
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    }
+  }
+}
+
+// A piece of a split unit: the row's unnormalised O, running max and row sum, column-major in
+// the slot (consecutive rows -> consecutive addresses), through L2.
+template <int D>
+UNSTEP_COLD_FN void write_piece(uint32_t tO, float *mine, int row, float m_run,
+                                         float l_run) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(tO + c * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) __stcg(mine + (c * 32 + e) * 128 + row, __uint_as_float(o[e]));
+  }
+  __stcg(mine + D * 128 + row, m_run);
+  __stcg(mine + D * 128 + 128 + row, l_run);
+  __threadfence();
+}
+
+// Scratch slot holding CTA c's piece of the tail unit whose first tile is t0 (tail-relative):
+// its first piece if its range starts inside the unit, else its second.
+__device__ __forceinline__ int piece_slot(const AttnParams &p, int c, long long t0) {
+  return 2 * c + (sk_lo(p, c) >= t0 ? 0 : 1);
+}
+
+// Merge the pieces of CTAs c_first..c_last for one row: rescale each to the common max,
+// sum, normalise, store.
+template <int D>
+UNSTEP_COLD_FN void merge_row(const AttnParams &p, int i, int row, long long t0,
+                                       int c_first, int c_last, __nv_bfloat16 *dst, bool live) {
+  constexpr int kTileFloats = D * 128 + 256;
+  __threadfence();
+  float M = -INFINITY;
+#pragma unroll 1
+  for (int c = c_first; c <= c_last; ++c) {
+    const float *src =
+        p.slots + static_cast<long long>(piece_slot(p, c, t0)) * p.slot_floats + i * kTileFloats;
+    M = fmaxf(M, __ldcg(src + D * 128 + row));
+  }
+  float Lsum = 0.f;
+#pragma unroll 1
+  for (int c = c_first; c <= c_last; ++c) {
+    const float *src =
+        p.slots + static_cast<long long>(piece_slot(p, c, t0)) * p.slot_floats + i * kTileFloats;
+    Lsum += __ldcg(src + D * 128 + 128 + row) * ex2_approx(__ldcg(src + D * 128 + row) - M);
+  }
+  const float inv = 1.f / Lsum;
+#pragma unroll 1
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int c = c_first; c <= c_last; ++c) {
+      const float *src =
+          p.slots + static_cast<long long>(piece_slot(p, c, t0)) * p.slot_floats + i * kTileFloats;
+      const float w = ex2_approx(__ldcg(src + D * 128 + row) - M);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a[e] = fmaf(w, __ldcg(src + (c8 * 8 + e) * 128 + row), a[e]);
+    }
+    if (live) {
+      uint4 v;
+      v.x = pack_bf16x2(a[0] * inv, a[1] * inv);
+      v.y = pack_bf16x2(a[2] * inv, a[3] * inv);
+      v.z = pack_bf16x2(a[4] * inv, a[5] * inv);
+      v.w = pack_bf16x2(a[6] * inv, a[7] * inv);
+      *reinterpret_cast<uint4 *>(dst + c8 * 8) = v;
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     window_attn_kernel(const __grid_constant__ CUtensorMap tmq,
@@ -160,7 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kSmemBar);
   uint64_t *q_full = bars;
-  uint64_t *full = bars + 1;
+  uint64_t *q_empty = bars + 1;
+  uint64_t *full = bars + 2;
   uint64_t *empty = full + NS;
   uint64_t *s_full = empty + NS;
   uint64_t *p_ready = s_full + 2;
@@ -168,18 +345,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain = o_done + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *merge_word = reinterpret_cast<volatile int *>(tmem_slot + 2);  // [2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = blockIdx.x % p.n_pairs;
-  const int bh = blockIdx.x / p.n_pairs;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-  const int q0 = pair * 256;
-  const bool has1 = q0 + 128 < p.L;
+  const int cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -203,145 +377,174 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, p.dev_error, p.wait_limit_ns};
   constexpr int E = UNSTEP_ERR_DEVICE_TIMEOUT;
+  const SkRange sk = sk_range(p, cta);
 
   if (warp >= 8) {
     regs_release<kRegsIo>();
-  if (warp == 8) {
-    // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmq);
-      tma_prefetch_desc(&tmk);
-      tma_prefetch_desc(&tmv);
-      const int nq = has1 ? 2 : 1;
-      mbar_arrive_expect_tx(q_full, nq * C::kTileBytes);
-      for (int t = 0; t < nq; ++t)
-        for (int c = 0; c < C::kBoxes; ++c)
-          tma_load_4d(smem + C::kSmemQ + t * C::kTileBytes + c * 16384, &tmq, q_full, c * 64, h,
-                      q0 + t * 128, b);
-      const int n_loads = 2 * p.n_tiles;
-      int issued = 0;
-      for (int n = 0; n < n_loads; ++n) {
-        const int s = n % NS;
-        const uint32_t r = static_cast<uint32_t>(n / NS);
-        if (!wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E)) break;
-        mbar_arrive_expect_tx(&full[s], C::kTileBytes);
-        int row, valid;
-        key_tile(p, n >> 1, row, valid);
-        const CUtensorMap *m = (n & 1) ? &tmv : &tmk;
-        for (int c = 0; c < C::kBoxes; ++c)
-          tma_load_3d(smem + C::kSmemKV + s * C::kTileBytes + c * 16384, m, &full[s], c * 64,
-                      row, bh);
-        issued = n + 1;
-      }
-      if (*abort_flag) {
-        // let every copy still in flight land before the CTA's shared memory is released
-        for (int n = max(0, issued - NS); n < issued; ++n)
-          wait_drain(&full[n % NS], static_cast<uint32_t>(n / NS) & 1u);
-        wait_drain(q_full, 0);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
-      const uint32_t sQ = smem_u32(smem + C::kSmemQ);
-      const uint32_t sKV = smem_u32(smem + C::kSmemKV);
-      // descriptors as 32-bit halves: the high half (stride offset, version, swizzle) is the
-      // same for every operand of a kind; only the start address in the low half moves
-      const uint32_t kHiK = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
-      const uint32_t kHiV = static_cast<uint32_t>(sdesc_sw128(0, 16384, 1024) >> 32);
-      const uint32_t loQ = static_cast<uint32_t>(sdesc_sw128(sQ, 16, 1024));
-      const uint32_t loK = static_cast<uint32_t>(sdesc_sw128(sKV, 16, 1024));
-      const uint32_t loV = static_cast<uint32_t>(sdesc_sw128(sKV, 16384, 1024));
-      auto qk = [&](int t, int s) {
-        const uint32_t dS = tmem + (t ? C::kTmS1 : C::kTmS0);
-        const uint32_t qa = loQ + static_cast<uint32_t>(t * (C::kTileBytes >> 4));
-        const uint32_t kb = loK + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          umma_ss(dS, f2u64(qa + off, kHiK), f2u64(kb + off, kHiK), kIdQK, kk > 0 ? 1u : 0u);
+    if (warp == 8) {
+      // -------------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+        int n = 0;   // K/V tiles issued
+        int nq = 0;  // Q loads issued
+        bool ok = true;
+        Seg sg;
+        for (int q = 0; ok && get_seg(p, cta, sk, q, sg); ++q) {
+          const UnitPos up = unit_pos(p, sg.u);
+          if (q > 0 && !(ok = wait_bounded(q_empty, static_cast<uint32_t>(q - 1) & 1u, g, E)))
+            break;
+          const int ntq = up.has1 ? 2 : 1;
+          mbar_arrive_expect_tx(q_full, ntq * C::kTileBytes);
+          for (int t = 0; t < ntq; ++t)
+            for (int c = 0; c < C::kBoxes; ++c)
+              tma_load_4d(smem + C::kSmemQ + t * C::kTileBytes + c * 16384, &tmq, q_full,
+                          c * 64, up.h, up.q0 + t * 128, up.b);
+          nq = q + 1;
+          for (int kt = sg.k0; ok && kt < sg.k1; ++kt) {
+            int row, valid;
+            key_tile(p, kt, row, valid);
+            for (int kv = 0; kv < 2; ++kv) {
+              const int s = n % NS;
+              const uint32_t r = static_cast<uint32_t>(n / NS);
+              if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
+              mbar_arrive_expect_tx(&full[s], C::kTileBytes);
+              const CUtensorMap *m = kv ? &tmv : &tmk;
+              for (int c = 0; c < C::kBoxes; ++c)
+                tma_load_3d(smem + C::kSmemKV + s * C::kTileBytes + c * 16384, m, &full[s],
+                            c * 64, row, up.bh);
+              ++n;
+            }
+          }
         }
-      };
-      auto pv = [&](int t, int s, bool acc) {
-        const uint32_t dO = tmem + (t ? C::kTmO1 : C::kTmO0);
-        const uint32_t aP = tmem + (t ? C::kTmS1 : C::kTmS0);
-        const uint32_t vb = loV + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(dO, aP + kk * 8, f2u64(vb + static_cast<uint32_t>(kk * (2048 >> 4)), kHiV),
-                  kIdPV, (acc || kk > 0) ? 1u : 0u);
-      };
-      auto wait_full = [&](int n) {
-        return wait_bounded(&full[n % NS], static_cast<uint32_t>(n / NS) & 1u, g, E);
-      };
-      bool ok = wait_bounded(q_full, 0, g, E) && wait_full(0);
-      if (ok) {
-        tc_fence_after();
-        qk(0, 0);
-        umma_commit(&s_full[0]);
-        if (has1) {
-          qk(1, 0);
-          umma_commit(&s_full[1]);
+        if (*abort_flag) {
+          // let every copy still in flight land before the CTA's shared memory is released
+          for (int k = max(0, n - NS); k < n; ++k)
+            wait_drain(&full[k % NS], static_cast<uint32_t>(k / NS) & 1u);
+          if (nq > 0) wait_drain(q_full, static_cast<uint32_t>(nq - 1) & 1u);
         }
-        umma_commit(&empty[0]);
       }
-      for (int j = 0; ok && j < p.n_tiles; ++j) {
-        const int nv = 2 * j + 1, nk = 2 * j + 2;
-        const int sv = nv % NS, sk = nk % NS;
-        const bool more = j + 1 < p.n_tiles;
-        const uint32_t ph = static_cast<uint32_t>(j) & 1u;
-        if (!(ok = wait_full(nv))) break;
-        if (!(ok = wait_bounded(&p_ready[0], ph, g, E))) break;
-        tc_fence_after();
-        pv(0, sv, j > 0);
-        umma_commit(&o_done[0]);
-        if (more) {
-          if (!(ok = wait_full(nk))) break;
+      __syncwarp();
+    } else if (warp == 9) {
+      // -------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
+        const uint32_t sQ = smem_u32(smem + C::kSmemQ);
+        const uint32_t sKV = smem_u32(smem + C::kSmemKV);
+        // descriptors as 32-bit halves: the high half (stride offset, version, swizzle) is the
+        // same for every operand of a kind; only the start address in the low half moves
+        const uint32_t kHiK = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
+        const uint32_t kHiV = static_cast<uint32_t>(sdesc_sw128(0, 16384, 1024) >> 32);
+        const uint32_t loQ = static_cast<uint32_t>(sdesc_sw128(sQ, 16, 1024));
+        const uint32_t loK = static_cast<uint32_t>(sdesc_sw128(sKV, 16, 1024));
+        const uint32_t loV = static_cast<uint32_t>(sdesc_sw128(sKV, 16384, 1024));
+        auto qk = [&](int t, int s) {
+          const uint32_t dS = tmem + (t ? C::kTmS1 : C::kTmS0);
+          const uint32_t qa = loQ + static_cast<uint32_t>(t * (C::kTileBytes >> 4));
+          const uint32_t kb = loK + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = static_cast<uint32_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            umma_ss(dS, f2u64(qa + off, kHiK), f2u64(kb + off, kHiK), kIdQK, kk > 0 ? 1u : 0u);
+          }
+        };
+        auto pv = [&](int t, int s, bool acc) {
+          const uint32_t dO = tmem + (t ? C::kTmO1 : C::kTmO0);
+          const uint32_t aP = tmem + (t ? C::kTmS1 : C::kTmS0);
+          const uint32_t vb = loV + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(dO, aP + kk * 8, f2u64(vb + static_cast<uint32_t>(kk * (2048 >> 4)), kHiV),
+                    kIdPV, (acc || kk > 0) ? 1u : 0u);
+        };
+        auto wait_full = [&](int k) {
+          return wait_bounded(&full[k % NS], static_cast<uint32_t>(k / NS) & 1u, g, E);
+        };
+        int n = 0;                  // K/V tiles consumed
+        uint32_t done0 = 0, done1 = 0;  // PVs issued per query tile (barrier phases)
+        bool ok = true;
+        Seg sg;
+        for (int q = 0; ok && get_seg(p, cta, sk, q, sg); ++q) {
+          const bool has1 = unit_pos(p, sg.u).has1;
+          const int ntl = sg.k1 - sg.k0;
+          if (!(ok = wait_bounded(q_full, static_cast<uint32_t>(q) & 1u, g, E))) break;
+          if (!(ok = wait_full(n))) break;
           tc_fence_after();
-          qk(0, sk);
+          qk(0, n % NS);
           umma_commit(&s_full[0]);
-        }
-        if (has1) {
-          if (!(ok = wait_bounded(&p_ready[1], ph, g, E))) break;
-          tc_fence_after();
-          pv(1, sv, j > 0);
-          umma_commit(&o_done[1]);
-        }
-        umma_commit(&empty[sv]);
-        if (more) {
           if (has1) {
-            qk(1, sk);
+            qk(1, n % NS);
             umma_commit(&s_full[1]);
           }
-          umma_commit(&empty[sk]);
+          umma_commit(&empty[n % NS]);
+          if (ntl == 1) umma_commit(q_empty);
+          for (int j = 0; j < ntl; ++j) {
+            const int nv = n + 2 * j + 1, nk = n + 2 * j + 2;
+            const bool more = j + 1 < ntl;
+            if (!(ok = wait_full(nv))) break;
+            if (!(ok = wait_bounded(&p_ready[0], done0 & 1u, g, E))) break;
+            tc_fence_after();
+            pv(0, nv % NS, j > 0);
+            umma_commit(&o_done[0]);
+            ++done0;
+            if (more) {
+              if (!(ok = wait_full(nk))) break;
+              tc_fence_after();
+              qk(0, nk % NS);
+              umma_commit(&s_full[0]);
+            }
+            if (has1) {
+              if (!(ok = wait_bounded(&p_ready[1], done1 & 1u, g, E))) break;
+              tc_fence_after();
+              pv(1, nv % NS, j > 0);
+              umma_commit(&o_done[1]);
+              ++done1;
+            }
+            umma_commit(&empty[nv % NS]);
+            if (more) {
+              if (has1) {
+                qk(1, nk % NS);
+                umma_commit(&s_full[1]);
+              }
+              umma_commit(&empty[nk % NS]);
+              if (j + 2 == ntl) umma_commit(q_empty);  // the segment's last QK^T is issued
+            }
+          }
+          n += 2 * ntl;
         }
+        // every MMA issued above has completed once `drain` flips
+        umma_commit(drain);
+        wait_drain(drain, 0);
       }
-      // every MMA issued above has completed once `drain` flips
-      umma_commit(drain);
-      wait_drain(drain, 0);
+      __syncwarp();
     }
-    __syncwarp();
-  }
   } else {
     regs_claim<kRegsSoftmax>();
     // ---------------------------------------------------------------- softmax + epilogue
     const int i = warp >> 2;          // query tile of this warpgroup
     const int wq = warp & 3;          // TMEM lane quarter
     const int row = threadIdx.x & 127;
-    if (i == 0 || has1) {
-      const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_base + (i ? C::kTmS1 : C::kTmS0);
-      const uint32_t tO = tmem + lane_base + (i ? C::kTmO1 : C::kTmO0);
-      const float scale = p.scale_log2;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (i ? C::kTmS1 : C::kTmS0);
+    const uint32_t tO = tmem + lane_base + (i ? C::kTmO1 : C::kTmO0);
+    const float scale = p.scale_log2;
+    constexpr int kTileFloats = D * 128 + 256;  // one query tile of a scratch slot
+    uint32_t cnt = 0;                           // key tiles this warpgroup has processed
+    bool ok = true;
+    Seg sg;
+    // Every segment is walked even after an abort (the work is skipped), so that the named
+    // barriers of the warpgroup are always reached by all of its threads.
+    for (int q = 0; get_seg(p, cta, sk, q, sg); ++q) {
+      const UnitPos up = unit_pos(p, sg.u);
+      if (i == 1 && !up.has1) continue;
+      const int ntl = sg.k1 - sg.k0;
       float m_run = -INFINITY, l_run = 0.f;
-      bool ok = true;
-      for (int j = 0; j < p.n_tiles; ++j) {
+      for (int j = 0; ok && j < ntl; ++j) {
         int krow, valid;
-        key_tile(p, j, krow, valid);
-        ok = __all_sync(kFull, wait_bounded(&s_full[i], static_cast<uint32_t>(j) & 1u, g, E));
+        key_tile(p, sg.k0 + j, krow, valid);
+        ok = __all_sync(kFull, wait_bounded(&s_full[i], cnt & 1u, g, E));
         if (!ok) break;
         tc_fence_after();
         uint32_t s[4][32];
@@ -364,8 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float f = ex2_approx(m_run - m_new);
           l_run *= f;
           m_run = m_new;
-          ok = __all_sync(kFull,
-                          wait_bounded(&o_done[i], static_cast<uint32_t>(j - 1) & 1u, g, E));
+          ok = __all_sync(kFull, wait_bounded(&o_done[i], (cnt - 1) & 1u, g, E));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -384,50 +586,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t acc[4] = {0, 0, 0, 0};
         if (!masked) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) exp_chunk<false>(s[c], c * 32, 128, sc2, nm2, acc, tS + c * 16);
+          for (int c = 0; c < 4; ++c)
+            exp_chunk<false>(s[c], c * 32, 128, sc2, nm2, acc, tS + c * 16);
         } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) exp_chunk<true>(s[c], c * 32, valid, sc2, nm2, acc, tS + c * 16);
+          for (int c = 0; c < 4; ++c)
+            exp_chunk<true>(s[c], c * 32, valid, sc2, nm2, acc, tS + c * 16);
         }
-        {
-          float a0, a1, b0, b1;
-          f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
-          (void)b0;
-          (void)b1;
-          l_run += a0 + a1;
-        }
+        float a0, a1;
+        f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+        l_run += a0 + a1;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_ready[i]);
+        ++cnt;
       }
-      if (ok) {
-        ok = __all_sync(kFull, wait_bounded(&o_done[i],
-                                            static_cast<uint32_t>(p.n_tiles - 1) & 1u, g, E));
+      if (ok) ok = __all_sync(kFull, wait_bounded(&o_done[i], (cnt - 1) & 1u, g, E));
+      if (ok) tc_fence_after();
+      const int l = up.q0 + i * 128 + row;
+      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
+                           ((static_cast<long long>(up.b) * p.L + l) * p.H + up.h) * D;
+      if (sg.slot < 0) {
+        if (ok) store_row<D>(tO, 1.f / l_run, dst, l < p.L);  // whole unit: normalise, store
+        continue;
       }
-      if (ok) {
-        tc_fence_after();
-        const float inv = 1.f / l_run;
-        const int l = q0 + i * 128 + row;
-        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
-                             ((static_cast<long long>(b) * p.L + l) * p.H + h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          if (l < p.L) {
-            uint32_t w[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
-                                 __uint_as_float(o[2 * e + 1]) * inv);
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      // piece of a split unit: leave it in the CTA's slot, count it, and merge if it was last
+      if (ok)
+        write_piece<D>(tO, p.slots + static_cast<long long>(sg.slot) * p.slot_floats +
+                               i * kTileFloats, row, m_run, l_run);
+      wg_sync(i);
+      const long long t0 = static_cast<long long>(sg.u - p.u_tail0) * p.n_tiles;
+      const int c_first = static_cast<int>(((t0 + 1) * p.g_sk - 1) / p.w_tail);
+      const int c_last = static_cast<int>(((t0 + p.n_tiles) * p.g_sk - 1) / p.w_tail);
+      if (threadIdx.x == 128 * i) {
+        int last = 0;
+        if (!*abort_flag) {
+          // count this piece; the count word carries the launch's epoch in its high bits, so a
+          // word left behind by an aborted launch is never mistaken for a current count
+          unsigned *ctr = p.counters + 2 * sg.u + i;
+          const unsigned ep = p.epoch << 8;
+          unsigned old = *reinterpret_cast<volatile unsigned *>(ctr), nw;
+          while (true) {
+            nw = ((old & 0xFFFFFF00u) == ep) ? old + 1 : (ep | 1u);
+            const unsigned seen = atomicCAS(ctr, old, nw);
+            if (seen == old) break;
+            old = seen;
           }
+          last = static_cast<int>(nw & 0xFFu) == c_last - c_first + 1;
+          if (last) atomicExch(ctr, 0u);
         }
+        merge_word[i] = last;
       }
+      wg_sync(i);
+      const bool merge = ok && merge_word[i] != 0;
+      wg_sync(i);  // merge_word is rewritten by the next piece
+      if (merge) merge_row<D>(p, i, row, t0, c_first, c_last, dst, l < p.L);
     }
   }
 
@@ -484,9 +697,8 @@ cudaError_t launch_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
     if (e != cudaSuccess) return e;
     if (dev < 64) __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
-  const long long grid = static_cast<long long>(p.B) * p.H * p.n_pairs;
-  if (grid < 1 || grid > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  window_attn_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmemAlloc, stream>>>(
+  if (p.grid < 1) return cudaErrorInvalidConfiguration;
+  window_attn_kernel<D><<<static_cast<unsigned>(p.grid), kThreads, C::kSmemAlloc, stream>>>(
       tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -79,6 +79,13 @@ typedef struct {
   int *slot_frame;  /* int32 [cap_frames]: frame held by each slot, -1 = empty */
   float *cos_sin;   /* fp32 coefficient tables, unstep_cache_table_bytes() bytes */
   int *dev_error;   /* int32 [1]: first device-side error, 0 = none */
+  /* optional attention scratch (caller-allocated, caller-owned; may be NULL): with it,
+   * unstep_window_attn balances its work over all SMs by splitting some (head, query) units
+   * along keys; without it, one CTA per unit.  unstep_attn_scratch_bytes() bytes, 16-byte
+   * aligned.  Several caches may share one scratch buffer if their attention calls never
+   * overlap on the GPU (e.g. they are issued on one stream). */
+  void *attn_scratch;
+  size_t attn_scratch_bytes;
   /* metadata (library-maintained; read-only for the caller) */
   int frames_written;    /* one past the newest frame written */
   int first_frame;       /* temporal position of the stream's first frame */
@@ -114,14 +121,20 @@ size_t unstep_cache_table_bytes(const unstep_cache_t *cache);
 /* Bytes of ONE of k_cache / v_cache for this shape (0 if invalid). */
 size_t unstep_cache_kv_bytes(const unstep_cache_t *cache);
 
+/* Bytes of the optional attention scratch for this shape on the CURRENT device (it depends on
+ * the device's SM count): per-(unit, query tile) counters plus two slots per SM of
+ * 2 x (D x 128 + 256) floats.  0 if the shape fields are invalid or no device is usable. */
+size_t unstep_attn_scratch_bytes(const unstep_cache_t *cache);
+
 /*
  * Validate the shape fields and pointers, compute the coefficient tables on the host in fp64,
- * round them to fp32 and copy them to cache->cos_sin; zero k_cache, v_cache and dev_error; set
- * every slot_frame entry to -1; reset the metadata.  Enqueued on `stream`; the table copy is from
- * pageable memory, so the call returns only after the copy has been staged.
+ * round them to fp32 and copy them to cache->cos_sin; zero k_cache, v_cache, dev_error and the
+ * scratch counters; set every slot_frame entry to -1; reset the metadata.  Enqueued on `stream`;
+ * the table copy is from pageable memory, so the call returns only after the copy has been
+ * staged.
  * Errors: ARG (NULL pointers, odd or negative split, split sum != D, cap_frames < 1,
- * max_pos_t < 1, theta <= 0), UNSUPPORTED (D not 64/128, sizes beyond 32-bit row indexing),
- * ALIGN, CUDA.
+ * max_pos_t < 1, theta <= 0, attn_scratch_bytes too small), UNSUPPORTED (D not 64/128, sizes
+ * beyond 32-bit row indexing), ALIGN, CUDA.
  */
 int unstep_cache_init(unstep_cache_t *cache, unstep_stream_t stream);
 

@@ -38,10 +38,11 @@ def gpu_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
-def make_cache(shape: W.LayerShape, cap: int, max_pos_t: int) -> binding.LayerCache:
+def make_cache(shape: W.LayerShape, cap: int, max_pos_t: int, use_scratch: bool = True,
+               scratch=None) -> binding.LayerCache:
     return binding.LayerCache(shape.B, shape.H, shape.D, shape.Hg, shape.Wg, shape.d_t,
                               shape.d_h, shape.d_w, cap_frames=cap, max_pos_t=max_pos_t,
-                              theta=shape.theta)
+                              theta=shape.theta, use_scratch=use_scratch, scratch=scratch)
 
 
 def make_oracle(shape: W.LayerShape, cap: int, heads=None) -> oracle.OracleLayer:

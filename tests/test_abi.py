@@ -65,6 +65,10 @@ def test_table_and_cache_sizes(L):
     c = _cache(s, 21)
     c.d_h = 41                 # odd block
     assert L.unstep_cache_table_bytes(ctypes.byref(c)) == 0
+    # the attention scratch depends on the device's SM count: 0 without a usable device
+    import torch
+    if not torch.cuda.is_available():
+        assert L.unstep_attn_scratch_bytes(ctypes.byref(_cache(s, 21))) == 0
 
 
 def test_init_rejects_bad_arguments_without_touching_the_device(L):

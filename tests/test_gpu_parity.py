@@ -19,8 +19,10 @@ from tests import parity as P
 pytestmark = pytest.mark.gpu
 
 
-def _run_stream(shape, cap, window, schedule, seed, check_cache=True, heads=None):
-    cache = P.make_cache(shape, cap, max_pos_t=max(f + n for f, n in schedule) + 1)
+def _run_stream(shape, cap, window, schedule, seed, check_cache=True, heads=None,
+                use_scratch=True):
+    cache = P.make_cache(shape, cap, max_pos_t=max(f + n for f, n in schedule) + 1,
+                         use_scratch=use_scratch)
     ol = P.make_oracle(shape, cap, heads=heads)
     hs = ol.heads
     worst = []
@@ -49,12 +51,18 @@ def _run_stream(shape, cap, window, schedule, seed, check_cache=True, heads=None
     return cache, ol, worst
 
 
-def test_tiny_workload():
+def _tiny(use_scratch=True):
     wl = W.WORKLOADS["tiny"]
     sched = [(wl.frame_idx(c), wl.shape.chunk_frames) for c in range(wl.chunks)]
-    cache, ol, errs = _run_stream(wl.shape, wl.cap, wl.window, sched, seed=1)
+    cache, ol, errs = _run_stream(wl.shape, wl.cap, wl.window, sched, seed=1,
+                                  use_scratch=use_scratch)
     assert cache.slot_frame.cpu().tolist() == [6, 7, 8, 3, 4, 5]
     assert max(e.rel_rms for e in errs) < 0.02
+
+
+@pytest.mark.parametrize("use_scratch", [True, False])
+def test_tiny_workload(use_scratch):
+    _tiny(use_scratch)
 
 
 @pytest.mark.parametrize("D,split", [(64, (24, 20, 20)), (128, (44, 42, 42))])
@@ -65,7 +73,9 @@ def test_tiny_workload():
     (3, 5, 3, 3, 3, 3, 100, 1, 2),    # tiny frames (15 tokens), late positions
     (11, 23, 3, 9, 9, 3, 0, 1, 2),    # 759 queries: 6 tiles incl. a partial, 1-3 key segments
 ])
-def test_streams_match_oracle(D, split, Hg, Wg, frames, cap, window, chunks, start, Bn, H):
+@pytest.mark.parametrize("use_scratch", [True, False])
+def test_streams_match_oracle(D, split, Hg, Wg, frames, cap, window, chunks, start, Bn, H,
+                              use_scratch):
     shape = W.LayerShape(B=Bn, H=H, D=D, Hg=Hg, Wg=Wg, d_t=split[0], d_h=split[1],
                          d_w=split[2], chunk_frames=frames)
     sched = []
@@ -74,7 +84,7 @@ def test_streams_match_oracle(D, split, Hg, Wg, frames, cap, window, chunks, sta
         sched.append((f, frames))
         if c == 1:
             sched.append((f, frames))  # re-forward of the same chunk (next denoising step)
-    _run_stream(shape, cap, window, sched, seed=D + Hg * 7 + cap)
+    _run_stream(shape, cap, window, sched, seed=D + Hg * 7 + cap, use_scratch=use_scratch)
 
 
 def _structured_v(shape, f0):
@@ -228,7 +238,7 @@ def test_bounded_wait_selftest_reports_timeout_and_context_survives():
     torch.cuda.synchronize()
     assert int(err.item()) == binding.UNSTEP_ERR_DEVICE_TIMEOUT
     # the context is still usable: a normal call runs and is correct
-    test_tiny_workload()
+    _tiny()
 
 
 def test_host_buffer_step_matches_device_path():
@@ -263,6 +273,7 @@ def test_exp2_polynomial_against_hardware_and_exact():
     assert rel_p < 1e-4, rel_p
     assert rel_m < 1e-5, rel_m
     assert (((yp - ym).abs() / ym).max().item()) < 1.1e-4
-    # below the clamp the polynomial returns 2^-125, never a negative or NaN value
-    y_low, _ = binding.selftest_exp2(torch.tensor([-200.0, -1e30], device="cuda"))
-    assert torch.all(y_low == torch.tensor(2.0 ** -125, device="cuda"))
+    # below the clamp the polynomial returns ~2^-125 (its value at -125), never 0, NaN or < 0
+    y_low, _ = binding.selftest_exp2(torch.tensor([-200.0, -1e30, -125.0], device="cuda"))
+    rel = (y_low.double().cpu() / 2.0 ** -125 - 1).abs()
+    assert torch.all(rel < 1e-4), y_low
