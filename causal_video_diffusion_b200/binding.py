@@ -24,6 +24,7 @@ UNSTEP_ERR_WINDOW = -5
 UNSTEP_ERR_UNSUPPORTED = -6
 UNSTEP_ERR_CUDA = -7
 UNSTEP_ERR_DEVICE_TIMEOUT = -8
+UNSTEP_ERR_SCRATCH_LIMIT = -9
 
 
 class unstep_cache_t(ctypes.Structure):
@@ -70,6 +71,9 @@ _SIGNATURES = {
                             ctypes.POINTER(unstep_window_plan_t)], ctypes.c_int),
     "unstep_window_attn": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t), ctypes.c_int,
                             ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "unstep_window_attn_noalloc": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t),
+                                    ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
+                                   ctypes.c_int),
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),

@@ -139,6 +139,8 @@ const char *unstep_status_string(int status) {
     case UNSTEP_ERR_UNSUPPORTED: return "unsupported head width or size";
     case UNSTEP_ERR_CUDA: return "CUDA runtime error";
     case UNSTEP_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
+    case UNSTEP_ERR_SCRATCH_LIMIT:
+      return "the call needs more scratch than the library's fixed device buffer holds";
     default: return "unknown status";
   }
 }
@@ -392,6 +394,99 @@ int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, v
   p.wait_limit_ns = unstep::kWaitLimitNs;
   if (unstep::launch_window_attn(D, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
+int unstep_window_attn_noalloc(const void *q, const unstep_cache_t *cache, int window,
+                               void *out, unstep_stream_t stream) {
+  int rc = check_ready(cache);
+  if (rc) return rc;
+  if (!q || !out) return UNSTEP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(out)) return UNSTEP_ERR_ALIGN;
+  unstep_window_plan_t plan;
+  rc = unstep_window_plan(cache, window, &plan);
+  if (rc) return rc;
+  const int D = cache->D, H = cache->H, B = cache->B;
+  const int tf = cache->Hg * cache->Wg;
+  const int L = cache->last_chunk_frames * tf;
+  const long long R = static_cast<long long>(cache->cap_frames) * tf;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  // the library's fixed buffer stands in for cache->attn_scratch (which is ignored here)
+  void *scratch = nullptr;
+  size_t capacity = 0;
+  if (unstep::static_attn_scratch(&scratch, &capacity) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  const int sms = device_sms();
+  if (sms <= 0) return UNSTEP_ERR_CUDA;
+  const int n_pairs = (L + 255) / 256;
+  const int U = B * H * n_pairs;
+  const size_t counter_bytes = unstep::attn_counter_bytes(U);
+  const size_t need = counter_bytes + 2ull * static_cast<size_t>(sms) *
+                                          unstep::attn_slot_floats(D) * sizeof(float);
+  if (need > capacity) return UNSTEP_ERR_SCRATCH_LIMIT;
+
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+    const cuuint64_t str[3] = {static_cast<cuuint64_t>(D) * 2,
+                               static_cast<cuuint64_t>(H) * D * 2,
+                               static_cast<cuuint64_t>(L) * H * D * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (!encode_bf16(&tq, q, 4, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(R),
+                                static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t str[2] = {static_cast<cuuint64_t>(D) * 2,
+                               static_cast<cuuint64_t>(R) * D * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!encode_bf16(&tk, cache->k_cache, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
+    if (!encode_bf16(&tv, cache->v_cache, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  unstep::AttnParams p{};
+  p.out = out;
+  p.dev_error = cache->dev_error;
+  p.B = B;
+  p.H = H;
+  p.L = L;
+  p.n_pairs = n_pairs;
+  p.n_units = U;
+  for (int s = 0; s < 2; ++s) {
+    p.seg_row[s] = plan.seg_row[s];
+    p.seg_len[s] = plan.seg_len[s];
+    p.seg_tiles[s] = (plan.seg_len[s] + 127) / 128;
+  }
+  p.n_tiles = p.seg_tiles[0] + p.seg_tiles[1];
+  p.div_pairs = unstep::make_fastdiv(static_cast<uint32_t>(p.n_pairs));
+  p.div_heads = unstep::make_fastdiv(static_cast<uint32_t>(H));
+  p.scale_log2 = static_cast<float>(1.4426950408889634073599 / std::sqrt(static_cast<double>(D)));
+  p.wait_limit_ns = unstep::kWaitLimitNs;
+  p.dp_waves = U / sms;
+  const int tail = U - p.dp_waves * sms;
+  p.u_tail0 = p.dp_waves * sms;
+  p.w_tail = static_cast<long long>(tail) * p.n_tiles;
+  long long gsk = tail > 0 ? static_cast<long long>(tail) * 8 : 0;
+  if (gsk > sms) gsk = sms;
+  if (gsk > p.w_tail) gsk = p.w_tail;
+  p.g_sk = static_cast<int>(gsk);
+  p.grid = p.dp_waves > 0 ? sms : p.g_sk;
+  p.counters = static_cast<unsigned *>(scratch);
+  p.slots = reinterpret_cast<float *>(static_cast<char *>(scratch) + counter_bytes);
+  p.slot_floats = static_cast<int>(unstep::attn_slot_floats(D));
+  p.epoch = next_epoch();
+  // the buffer keeps whatever the previous call left in it: the counts must start at zero
+  if (cudaMemsetAsync(scratch, 0, counter_bytes, st) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  if (unstep::launch_window_attn(D, tq, tk, tv, p, st) != cudaSuccess) {
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
   }

@@ -92,6 +92,13 @@ cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorM
 
 cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cudaStream_t stream);
 
+// Size of the library's fixed device scratch buffer (see unstep_window_attn_noalloc).
+constexpr size_t kStaticScratchBytes = 48ull << 20;
+
+// Device address and size of that buffer on the current device; the first call on a device
+// looks the address up (cudaGetSymbolAddress with the device current) and caches it.
+cudaError_t static_attn_scratch(void **ptr, size_t *bytes);
+
 cudaError_t launch_exp2_selftest(const float *x, float *y_poly, float *y_mufu, int n,
                                  cudaStream_t stream);
 

@@ -29,6 +29,8 @@
 // lets in-flight TMA copies and MMAs land, frees TMEM and exits.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "../../include/unstep.h"
 #include "internal.h"
 #include "sm100.cuh"
@@ -711,6 +713,38 @@ cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorM
   if (D == 128) return launch_d<128>(tmap_q, tmap_k, tmap_v, p, stream);
   if (D == 64) return launch_d<64>(tmap_q, tmap_k, tmap_v, p, stream);
   return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Fixed device scratch for callers that cannot allocate device memory.
+//
+// Some callers have no way to call cudaMalloc: code that runs inside a framework or allocator
+// that owns every device allocation, or a process that must not grow its device footprint once
+// it has started.  For them the attention's split-unit scratch (per-unit counts and the pieces'
+// partial results) lives in this buffer, which is part of the library image: every device that
+// loads the library holds kStaticScratchBytes of it until the process exits.  Host code cannot
+// use the symbol's name as a device address (it names a host-side stand-in), so the address is
+// looked up once per device, with that device current, and passed to the kernel.
+// ---------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_attn_static_scratch[kStaticScratchBytes];
+
+cudaError_t static_attn_scratch(void **ptr, size_t *bytes) {
+  static std::mutex mu;
+  static void *addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_attn_static_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = a;
+  }
+  *ptr = addr[dev];
+  *bytes = kStaticScratchBytes;
+  return cudaSuccess;
 }
 
 cudaError_t launch_exp2_selftest(const float *x, float *y_poly, float *y_mufu, int n,

@@ -55,7 +55,8 @@ enum {
   UNSTEP_ERR_WINDOW = -5,         /* window outside [chunk frames, cap_frames], or empty cache */
   UNSTEP_ERR_UNSUPPORTED = -6,    /* D not 64/128, or a size beyond the kernels' index range */
   UNSTEP_ERR_CUDA = -7,           /* a CUDA runtime call failed (launch, copy, memset) */
-  UNSTEP_ERR_DEVICE_TIMEOUT = -8  /* a kernel gave up waiting (reported by the device word) */
+  UNSTEP_ERR_DEVICE_TIMEOUT = -8, /* a kernel gave up waiting (reported by the device word) */
+  UNSTEP_ERR_SCRATCH_LIMIT = -9   /* unstep_window_attn_noalloc: call too large for its buffer */
 };
 
 /*
@@ -186,6 +187,30 @@ int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_pl
  */
 int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
                        unstep_stream_t stream);
+
+/*
+ * unstep_window_attn for callers that cannot allocate device memory.
+ * No counterpart in the paper.  Some callers have no way to call cudaMalloc (code running under
+ * a framework or allocator that owns every device allocation, or a process whose device
+ * footprint must not grow after start-up), so they cannot provide cache->attn_scratch.  This
+ * call computes exactly what unstep_window_attn computes, with the same load-balanced schedule,
+ * but keeps its scratch in a buffer that is part of the library itself: 48 MiB of device memory
+ * (a file-scope __device__ array) that every GPU which loads the library holds until the process
+ * exits.  cache->attn_scratch is ignored.  The call allocates nothing and calls no allocating
+ * routine.
+ *   - The first call on a device looks up the buffer's device address (with that device current)
+ *     and caches it; make that first call before any stream capture.
+ *   - Every call on a device uses the same buffer and zeroes the part that must start at zero
+ *     (its counters) on `stream` before the kernel.  Calls whose work overlaps on the GPU (two
+ *     streams, two threads) race on the buffer: issue them in one stream order.
+ *   - Limit: the buffer must hold 2 x (SM count) slots of 2 x (D x 128 + 256) floats plus
+ *     8 bytes per (head, 256-query) unit; on a 148-SM B200 with D = 128 that is 37.6 MiB plus the
+ *     counters, which covers up to about 1.3 million units.  A larger call returns
+ *     UNSTEP_ERR_SCRATCH_LIMIT without doing anything.
+ * Errors: those of unstep_window_attn, plus SCRATCH_LIMIT.
+ */
+int unstep_window_attn_noalloc(const void *q, const unstep_cache_t *cache, int window,
+                               void *out, unstep_stream_t stream);
 
 /*
  * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported
