@@ -276,6 +276,79 @@ class LayerCache:
         return out_h
 
 
+class HostStepPipeline:
+    """Layer steps fed from pinned host memory, with copies overlapped with compute.
+
+    Step i copies its q, k, v host->device on one copy stream, runs ``rope_kv_append`` and
+    ``window_attn`` on the compute stream, and copies its output device->host on a second copy
+    stream; two sets of device buffers alternate, so step i+1's input copy and step i-1's output
+    copy run while step i computes.  Every step still moves all of its inputs and its output
+    across the host link.
+    """
+
+    def __init__(self, cache: LayerCache, device=None):
+        c = cache.c
+        dev = cache.device if device is None else torch.device(device)
+        self.cache = cache
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        self.compute = torch.cuda.Stream(device=dev)
+        self.device = dev
+        self.sets = []
+        self.c = c
+
+    def _bufs(self, L: int):
+        c = self.c
+        if not self.sets or self.sets[0]["q"].shape[1] != L:
+            self.sets = [{n: torch.empty((c.B, L, c.H, c.D), dtype=torch.bfloat16,
+                                         device=self.device) for n in ("q", "k", "v", "out")}
+                         for _ in range(2)]
+        return self.sets
+
+    def run(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, frame_idx: int,
+            frames: int, window: int, out_h: torch.Tensor, steps: int) -> float:
+        """Run ``steps`` steps (the same chunk re-forwarded; inputs copied every step) and return
+        the device time in ms from the first input copy to the last output copy."""
+        sets = self._bufs(q_h.shape[1])
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        start, end = ev(), ev()
+        in_ready = [None, None]
+        computed = [None, None]
+        out_done = [None, None]
+        torch.cuda.synchronize(self.device)
+        start.record(self.h2d)
+        for i in range(steps):
+            b = i & 1
+            bufs = sets[b]
+            with torch.cuda.stream(self.h2d):
+                if computed[b] is not None:
+                    self.h2d.wait_event(computed[b])   # the set's previous step is done with it
+                bufs["q"].copy_(q_h, non_blocking=True)
+                bufs["k"].copy_(k_h, non_blocking=True)
+                bufs["v"].copy_(v_h, non_blocking=True)
+                in_ready[b] = ev()
+                in_ready[b].record(self.h2d)
+            with torch.cuda.stream(self.compute):
+                self.compute.wait_event(in_ready[b])
+                if out_done[b] is not None:
+                    self.compute.wait_event(out_done[b])  # its output has left the device
+                self.cache.rope_kv_append(bufs["q"], bufs["k"], bufs["v"], frame_idx, frames,
+                                          stream=self.compute)
+                self.cache.window_attn(bufs["q"], window, out=bufs["out"], stream=self.compute)
+                computed[b] = ev()
+                computed[b].record(self.compute)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(computed[b])
+                out_h.copy_(bufs["out"], non_blocking=True)
+                out_done[b] = ev()
+                out_done[b].record(self.d2h)
+        self.h2d.wait_stream(self.d2h)
+        self.h2d.wait_stream(self.compute)
+        end.record(self.h2d)
+        end.synchronize()
+        return start.elapsed_time(end)
+
+
 def selftest_wait_timeout(dev_error: torch.Tensor, limit_ns: int,
                           stream: Optional[torch.cuda.Stream] = None) -> None:
     _check(lib().unstep_selftest_wait_timeout(_dev_ptr(dev_error, "dev_error"), int(limit_ns),

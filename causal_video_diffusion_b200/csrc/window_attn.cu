@@ -55,11 +55,15 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * 168, "registe
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
+#ifndef UNSTEP_KV_STAGES
+#define UNSTEP_KV_STAGES 4
+#endif
+
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;                // 128-byte swizzle boxes per row
   static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16
-  static constexpr int kStages = 4;                    // K/V ring stages
+  static constexpr int kStages = UNSTEP_KV_STAGES;     // K/V ring stages
   static constexpr int kSmemQ = 0;
   static constexpr int kSmemKV = 2 * kTileBytes;
   static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;

@@ -277,3 +277,27 @@ def test_exp2_polynomial_against_hardware_and_exact():
     y_low, _ = binding.selftest_exp2(torch.tensor([-200.0, -1e30, -125.0], device="cuda"))
     rel = (y_low.double().cpu() / 2.0 ** -125 - 1).abs()
     assert torch.all(rel < 1e-4), y_low
+
+
+def test_host_pipeline_matches_device_path():
+    """The overlapped host pipeline produces the same output as the plain device calls."""
+    wl = W.WORKLOADS["tiny"]
+    s = wl.shape
+    a = P.make_cache(s, wl.cap, 9)
+    b = P.make_cache(s, wl.cap, 9)
+    for c in range(2):
+        q, k, v = W.gen_qkv(60 + c, s)
+        for cache in (a, b):
+            qd = q.cuda()
+            cache.rope_kv_append(qd, k.cuda(), v.cuda(), 3 * c, 3)
+            cache.window_attn(qd, 6)
+    q, k, v = W.gen_qkv(70, s)
+    qd = q.cuda()
+    a.rope_kv_append(qd, k.cuda(), v.cuda(), 3, 3)   # re-forward of the latest chunk
+    want = a.window_attn(qd, 6).cpu()
+    out_h = torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16).pin_memory()
+    ms = binding.HostStepPipeline(b).run(q.pin_memory(), k.pin_memory(), v.pin_memory(), 3, 3, 6,
+                                          out_h, steps=5)
+    assert ms > 0
+    assert torch.equal(out_h, want)
+    assert b.device_error() == 0
