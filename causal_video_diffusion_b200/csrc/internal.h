@@ -10,25 +10,6 @@ namespace unstep {
 // Default limit of every device-side wait: no legitimate wait of these kernels lasts this long.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-struct RopeAppendParams {
-  const void *k;
-  const void *v;
-  void *q;
-  void *k_cache;
-  void *v_cache;
-  int *slot_frame;
-  const float2 *tab_t;  // [max_pos_t][d_t/2]
-  const float2 *tab_h;  // [Hg][d_h/2]
-  const float2 *tab_w;  // [Wg][d_w/2]
-  int B, L, H, D;
-  int Hg, Wg, Tf;
-  int half_t, half_h, half_w;  // pairs per block
-  int frame_idx, frames, cap;
-  int rows;  // cap * Tf
-};
-
-cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream);
-
 // Division by a run-time invariant d by multiply-high (Granlund & Montgomery, "Division by
 // invariant integers using multiplication", PLDI 1994): with l = ceil(log2 d) and
 // m = floor(2^32 (2^l - d) / d) + 1, x / d = (umulhi(x, m) + x) >> l for 0 <= x < 2^31.
@@ -48,6 +29,30 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv &f) {
   return (__umulhi(x, f.m) + x) >> f.l;
 }
 #endif
+
+struct RopeAppendParams {
+  const void *k;
+  const void *v;
+  void *q;
+  void *k_cache;
+  void *v_cache;
+  int *slot_frame;
+  const float2 *tab_t;  // [max_pos_t][d_t/2]
+  const float2 *tab_h;  // [Hg][d_h/2]
+  const float2 *tab_w;  // [Wg][d_w/2]
+  int B, L, H, D;
+  int Hg, Wg, Tf;
+  int half_t, half_h, half_w;  // pairs per block
+  int frame_idx, frames, cap;
+  int rows;       // cap * Tf
+  int slot0;      // frame_idx mod cap
+  FastDiv div_h;  // by H
+  FastDiv div_l;  // by L
+  FastDiv div_tf; // by Tf
+  FastDiv div_wg; // by Wg
+};
+
+cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream);
 
 struct AttnParams {
   void *out;         // bf16 [B][L][H][D]

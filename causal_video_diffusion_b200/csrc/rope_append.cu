@@ -14,7 +14,10 @@ namespace unstep {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kItemsPerThread = 2;  // independent 16-byte vectors in flight per thread
+#ifndef UNSTEP_ROPE_ITEMS
+#define UNSTEP_ROPE_ITEMS 1
+#endif
+constexpr int kItemsPerThread = UNSTEP_ROPE_ITEMS;  // independent 16-byte vectors per thread
 
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
   uint4 r;
@@ -50,34 +53,37 @@ struct Item {
   float2 cs[4];      // cos/sin of its 4 channel pairs
 };
 
+// Where item `it` (one 8-channel vector of one (stream, token, head)) lives, and its coefficients.
+// All index arithmetic is 32-bit (items < 2^31, checked on the host) with multiply-high division.
 template <int D>
-__device__ __forceinline__ void locate(const RopeAppendParams &p, long long it, Item &m) {
-  constexpr int V = D / 8;  // 16-byte vectors per head row
-  const int c8 = static_cast<int>(it % V);
-  const long long r = it / V;  // (b*L + l)*H + h
-  const int h = static_cast<int>(r % p.H);
-  const long long bl = r / p.H;
-  const int l = static_cast<int>(bl % p.L);
-  const int b = static_cast<int>(bl / p.L);
-  const int i = l / p.Tf;
-  const int tok = l - i * p.Tf;
-  const int y = tok / p.Wg;
-  const int x = tok - y * p.Wg;
-  const int f = p.frame_idx + i;
-  const int slot = f % p.cap;
-  m.e = it * 8;
+__device__ __forceinline__ void locate(const RopeAppendParams &p, uint32_t it, Item &m) {
+  constexpr int kLogV = (D == 128) ? 4 : 3;  // 16-byte vectors per head row: D / 8
+  const uint32_t c8 = it & ((1u << kLogV) - 1);
+  const uint32_t r = it >> kLogV;             // (b*L + l)*H + h
+  const uint32_t bl = fdiv(r, p.div_h);
+  const uint32_t h = r - bl * static_cast<uint32_t>(p.H);
+  const uint32_t b = fdiv(bl, p.div_l);
+  const uint32_t l = bl - b * static_cast<uint32_t>(p.L);
+  const uint32_t i = fdiv(l, p.div_tf);
+  const uint32_t tok = l - i * static_cast<uint32_t>(p.Tf);
+  const uint32_t y = fdiv(tok, p.div_wg);
+  const uint32_t x = tok - y * static_cast<uint32_t>(p.Wg);
+  const int f = p.frame_idx + static_cast<int>(i);
+  int slot = p.slot0 + static_cast<int>(i);   // i < frames <= cap: one wrap at most
+  if (slot >= p.cap) slot -= p.cap;
+  m.e = static_cast<long long>(it) * 8;
   m.ce = ((static_cast<long long>(b) * p.H + h) * p.rows + static_cast<long long>(slot) * p.Tf +
           tok) * D + c8 * 8;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const int pr = c8 * 4 + u;  // channel pair index
+    const int pr = static_cast<int>(c8) * 4 + u;  // channel pair index
     const float2 *src;
     if (pr < p.half_t) {
-      src = p.tab_t + static_cast<long long>(f) * p.half_t + pr;
+      src = p.tab_t + f * p.half_t + pr;
     } else if (pr < p.half_t + p.half_h) {
-      src = p.tab_h + y * p.half_h + (pr - p.half_t);
+      src = p.tab_h + static_cast<int>(y) * p.half_h + (pr - p.half_t);
     } else {
-      src = p.tab_w + x * p.half_w + (pr - p.half_t - p.half_h);
+      src = p.tab_w + static_cast<int>(x) * p.half_w + (pr - p.half_t - p.half_h);
     }
     m.cs[u] = __ldg(src);
   }
@@ -85,9 +91,8 @@ __device__ __forceinline__ void locate(const RopeAppendParams &p, long long it, 
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppendParams p,
-                                                                   long long n_items) {
-  const long long base =
-      static_cast<long long>(blockIdx.x) * (kThreads * kItemsPerThread) + threadIdx.x;
+                                                                   uint32_t n_items) {
+  const uint32_t base = blockIdx.x * (kThreads * kItemsPerThread) + threadIdx.x;
   if (blockIdx.x == 0 && threadIdx.x < p.frames) {
     const int f = p.frame_idx + threadIdx.x;
     p.slot_frame[f % p.cap] = f;
@@ -97,7 +102,7 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
   bool live[kItemsPerThread];
 #pragma unroll
   for (int u = 0; u < kItemsPerThread; ++u) {
-    const long long it = base + u * kThreads;
+    const uint32_t it = base + u * kThreads;
     live[u] = it < n_items;
     if (live[u]) {
       locate<D>(p, it, m[u]);
@@ -128,14 +133,21 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
 
 cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream) {
   const long long n_items = static_cast<long long>(p.B) * p.L * p.H * (p.D / 8);
+  if (n_items >= (1ll << 31) - kThreads * kItemsPerThread) return cudaErrorInvalidConfiguration;
+  RopeAppendParams q = p;
+  q.slot0 = p.frame_idx % p.cap;
+  q.div_h = make_fastdiv(static_cast<uint32_t>(p.H));
+  q.div_l = make_fastdiv(static_cast<uint32_t>(p.L));
+  q.div_tf = make_fastdiv(static_cast<uint32_t>(p.Tf));
+  q.div_wg = make_fastdiv(static_cast<uint32_t>(p.Wg));
   const long long per_block = kThreads * kItemsPerThread;
   long long blocks = (n_items + per_block - 1) / per_block;
   if (blocks < 1) blocks = 1;
-  if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  const uint32_t n = static_cast<uint32_t>(n_items);
   if (p.D == 128) {
-    rope_kv_append_kernel<128><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(p, n_items);
+    rope_kv_append_kernel<128><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(q, n);
   } else if (p.D == 64) {
-    rope_kv_append_kernel<64><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(p, n_items);
+    rope_kv_append_kernel<64><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(q, n);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -189,3 +189,26 @@ def test_exp2_polynomial_coefficients_match_their_derivation():
     c = np.float32(m.remez_exp2())
     assert np.allclose(consts, c, rtol=0, atol=1e-7)
     assert m.max_rel_err(c) < 8e-5
+
+
+def test_multiply_high_division_method():
+    """The kernels divide by run-time invariants with Granlund & Montgomery's multiply-high
+    method (m = floor(2^32 (2^l - d) / d) + 1, l = ceil(log2 d), q = (umulhi(x, m) + x) >> l);
+    check it against exact division over the dividend range they use (x < 2^31)."""
+    rng = np.random.default_rng(9)
+    ds = [1, 2, 3, 5, 7, 12, 19, 21, 24, 52, 1560, 4680, 65535, 65536, 999983, 2 ** 20 + 1]
+    ds += [int(d) for d in rng.integers(1, 2 ** 24, size=40)]
+    xs = np.concatenate([rng.integers(0, 2 ** 31, size=4000, dtype=np.int64),
+                         np.array([0, 1, 2 ** 31 - 1, 2 ** 31 - 2], dtype=np.int64)])
+    for d in ds:
+        l = 0
+        while (1 << l) < d:
+            l += 1
+        m = ((1 << 32) * ((1 << l) - d)) // d + 1
+        assert m < (1 << 32)
+        xs_d = np.concatenate([xs, np.arange(0, 4 * d, max(1, d // 3), dtype=np.int64)[:2000],
+                               (np.arange(1, 200, dtype=np.int64) * d - 1)])
+        xs_d = xs_d[(xs_d >= 0) & (xs_d < 2 ** 31)]
+        hi = (xs_d.astype(object) * m) >> 32
+        q = np.array([(int(h) + int(x)) >> l for h, x in zip(hi, xs_d)], dtype=np.int64)
+        assert np.array_equal(q, xs_d // d), d
