@@ -74,6 +74,12 @@ _SIGNATURES = {
     "unstep_window_attn_noalloc": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t),
                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
                                    ctypes.c_int),
+    "unstep_gemm_bf16": ([ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                          ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                          ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "unstep_lowrank_linear": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                               ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),
@@ -347,6 +353,57 @@ class HostStepPipeline:
         end.record(self.h2d)
         end.synchronize()
         return start.elapsed_time(end)
+
+
+def _err_word(dev_error: Optional[torch.Tensor], like: torch.Tensor) -> torch.Tensor:
+    if dev_error is None:
+        dev_error = torch.zeros(1, dtype=torch.int32, device=like.device)
+    return dev_error
+
+
+def gemm_bf16(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None,
+              dev_error: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """out[M][N] = a[M][K] @ b[N][K]^T on the tensor cores (bf16 in, fp32 accumulate, bf16 out)."""
+    for t, n in ((a, "a"), (b, "b")):
+        if t.dtype != torch.bfloat16 or t.dim() != 2:
+            raise ValueError(f"{n} must be a 2-D bfloat16 tensor")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b disagree on K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    err = _err_word(dev_error, a)
+    _check(lib().unstep_gemm_bf16(_dev_ptr(a, "a"), K, _dev_ptr(b, "b"), K, _dev_ptr(out, "out"),
+                                  N, M, N, K, _dev_ptr(err, "dev_error"), _stream_handle(stream)),
+           "unstep_gemm_bf16")
+    return out
+
+
+def lowrank_linear(x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
+                   t: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                   dev_error: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """y = (x @ w1^T) @ w2^T: a linear layer through its truncated-SVD factors."""
+    M, d_in = x.shape
+    rank = w1.shape[0]
+    d_out = w2.shape[0]
+    if w1.shape[1] != d_in or w2.shape[1] != rank:
+        raise ValueError("factor shapes do not chain")
+    for tt, n in ((x, "x"), (w1, "w1"), (w2, "w2")):
+        if tt.dtype != torch.bfloat16:
+            raise ValueError(f"{n} must be bfloat16")
+    if t is None:
+        t = torch.empty((M, rank), dtype=torch.bfloat16, device=x.device)
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.bfloat16, device=x.device)
+    err = _err_word(dev_error, x)
+    _check(lib().unstep_lowrank_linear(_dev_ptr(x, "x"), _dev_ptr(w1, "w1"), _dev_ptr(w2, "w2"),
+                                       _dev_ptr(t, "t"), _dev_ptr(y, "y"), M, d_in, rank, d_out,
+                                       _dev_ptr(err, "dev_error"), _stream_handle(stream)),
+           "unstep_lowrank_linear")
+    return y
 
 
 def selftest_wait_timeout(dev_error: torch.Tensor, limit_ns: int,

@@ -493,6 +493,41 @@ int unstep_window_attn_noalloc(const void *q, const unstep_cache_t *cache, int w
   return UNSTEP_OK;
 }
 
+int unstep_gemm_bf16(const void *a, int lda, const void *b, int ldb, void *c, int ldc, int M,
+                     int N, int K, int *dev_error, unstep_stream_t stream) {
+  if (!a || !b || !c || !dev_error) return UNSTEP_ERR_ARG;
+  if (M < 1 || N < 1 || K < 1) return UNSTEP_ERR_SHAPE;
+  if ((N & 7) || (K & 7) || (lda & 7) || (ldb & 7) || (ldc & 7) || lda < K || ldb < K || ldc < N)
+    return UNSTEP_ERR_SHAPE;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c)) return UNSTEP_ERR_ALIGN;
+  CUtensorMap ta, tb;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t str[1] = {static_cast<cuuint64_t>(lda) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!encode_bf16(&ta, a, 2, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+    const cuuint64_t str[1] = {static_cast<cuuint64_t>(ldb) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!encode_bf16(&tb, b, 2, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  if (unstep::launch_gemm_bf16_tn(ta, tb, c, M, N, K, ldc, dev_error,
+                                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
+int unstep_lowrank_linear(const void *x, const void *w1, const void *w2, void *t, void *y, int M,
+                          int d_in, int rank, int d_out, int *dev_error, unstep_stream_t stream) {
+  int rc = unstep_gemm_bf16(x, d_in, w1, d_in, t, rank, M, rank, d_in, dev_error, stream);
+  if (rc) return rc;
+  return unstep_gemm_bf16(t, rank, w2, rank, y, d_out, M, d_out, rank, dev_error, stream);
+}
+
 int unstep_get_device_error(const unstep_cache_t *cache, unstep_stream_t stream) {
   if (!cache || !cache->dev_error) return UNSTEP_ERR_ARG;
   int v = 0;

@@ -97,6 +97,11 @@ cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorM
 
 cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cudaStream_t stream);
 
+// C[M][N] (ldc) = A[M][K] * B[N][K]^T, bf16, fp32 accumulation; tma: 2D (K, M) box (64, 128),
+// tmb: 2D (K, N) box (64, 128), both 128B swizzle.
+cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
+                                int N, int K, int ldc, int *dev_error, cudaStream_t stream);
+
 // Size of the library's fixed device scratch buffer (see unstep_window_attn_noalloc).
 constexpr size_t kStaticScratchBytes = 48ull << 20;
 

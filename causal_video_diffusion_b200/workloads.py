@@ -139,3 +139,23 @@ def from_bits(a) -> torch.Tensor:
     """A bf16 CPU tensor from a numpy uint16 array of bit patterns."""
     import numpy as np
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+# the truncated-SVD projections of the same layer: 1536 = 12 heads x 128 channels
+MODEL_DIM = 12 * 128
+
+
+def gen_weight(seed: int, d_out: int, d_in: int) -> torch.Tensor:
+    """A synthetic fp32 projection weight [d_out][d_in], i.i.d. N(0, 1/d_in) (unit-variance
+    outputs for unit-variance inputs), from a seeded CPU generator."""
+    g = torch.Generator()
+    g.manual_seed(int(seed))
+    return torch.randn((d_out, d_in), generator=g, dtype=torch.float32) / (d_in ** 0.5)
+
+
+def gen_act(seed: int, rows: int, cols: int, device: str = "cpu") -> torch.Tensor:
+    """bf16 activations [rows][cols] from N(0, 1) fp32 draws."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return torch.randn((rows, cols), generator=g, dtype=torch.float32,
+                       device=device).to(torch.bfloat16)

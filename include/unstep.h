@@ -213,6 +213,28 @@ int unstep_window_attn_noalloc(const void *q, const unstep_cache_t *cache, int w
                                void *out, unstep_stream_t stream);
 
 /*
+ * Dense GEMM on the tensor cores: C[M][N] = A[M][K] * B[N][K]^T (both operands K-contiguous,
+ * nn.Linear's weight layout for B), bf16 in, fp32 accumulation, bf16 RNE out.  Row strides
+ * lda, ldb, ldc in elements.  N, K and the strides must be multiples of 8 (16-byte rows for TMA);
+ * M, N, K otherwise arbitrary (ragged tiles are zero-filled and not stored).  A device-side wait
+ * that runs out sets *dev_error.  Errors: ARG, SHAPE, ALIGN, CUDA.
+ */
+int unstep_gemm_bf16(const void *a, int lda, const void *b, int ldb, void *c, int ldc, int M,
+                     int N, int K, int *dev_error, unstep_stream_t stream);
+
+/*
+ * Truncated-SVD projection (UnStep, abstract and Figure 11 / Table 5: truncated SVD of the
+ * attention's value and output projections, rank retention 0.92): a linear layer y = x W^T with
+ * W [d_out][d_in] ~ U_r S_r V_r^T evaluated through its rank-`rank` factors,
+ *   t = x w1^T   (w1 = (V_r S_r)^T, bf16 [rank][d_in]),   y = t w2^T   (w2 = U_r, bf16 [d_out][rank]),
+ * as two unstep_gemm_bf16 calls.  x: [M][d_in]; t: caller scratch [M][rank]; y: [M][d_out].
+ * rank, d_in and d_out must be multiples of 8 (pad the factors with zero rows/columns: the
+ * product is unchanged).  Errors: those of unstep_gemm_bf16.
+ */
+int unstep_lowrank_linear(const void *x, const void *w1, const void *w2, void *t, void *y, int M,
+                          int d_in, int rank, int d_out, int *dev_error, unstep_stream_t stream);
+
+/*
  * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported
  * an error); CUDA if the copy or the synchronisation itself failed.
  */

@@ -318,3 +318,28 @@ class OracleLayer:
     def stored_k(self) -> np.ndarray:
         """The rotated keys as a bf16 cache holds them (RNE of the fp64 rotation)."""
         return f64_to_bf16(self.K)
+
+
+# --------------------------------------------------------------------------------------------
+# Truncated-SVD projections (abstract; Figure 11 / Table 5: V/O rank retention 0.92)
+# --------------------------------------------------------------------------------------------
+
+def matmul_bt(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
+    """C = A B^T in fp64 from bf16 bit patterns (A [M][K], B [N][K])."""
+    return bf16_to_f64(a_bits) @ bf16_to_f64(b_bits).T
+
+
+def lowrank_linear(x_bits, w1_bits, w2_bits, round_t: bool = False) -> np.ndarray:
+    """y = (x w1^T) w2^T in fp64; with round_t the rank-space product is rounded to bf16 (RNE)
+    first, as a bf16 intermediate buffer holds it."""
+    t = matmul_bt(x_bits, w1_bits)
+    if round_t:
+        t = bf16_to_f64(f64_to_bf16(t))
+    return t @ bf16_to_f64(w2_bits).T
+
+
+def svd_truncate(W: np.ndarray, rank: int):
+    """Factors of the rank-`rank` truncation of W [d_out][d_in] by numpy's SVD:
+    (w1 = (V_r S_r)^T [rank][d_in], w2 = U_r [d_out][rank], singular values)."""
+    U, S, Vh = np.linalg.svd(np.asarray(W, dtype=np.float64), full_matrices=False)
+    return (S[:rank, None] * Vh[:rank]), U[:, :rank], S

@@ -1,0 +1,73 @@
+"""The tensor-core GEMM and the truncated-SVD projections against the fp64 oracle (GPU)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_video_diffusion_b200 import binding
+from causal_video_diffusion_b200 import lowrank
+from causal_video_diffusion_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _rel_errors(got, want):
+    d = np.abs(got - want)
+    rms = float(np.sqrt(np.mean(want ** 2))) or 1.0
+    return float(d.max()) / rms, float(d.mean()) / rms
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 8, 8), (300, 136, 1416), (4680, 1416, 1536),
+                                   (257, 520, 72), (129, 264, 200)])
+def test_gemm_matches_oracle(M, N, K):
+    a = W.gen_act(M * 7 + 1, M, K)
+    b = W.gen_act(N * 11 + 2, N, K)
+    got = binding.gemm_bf16(a.cuda(), b.cuda()).cpu().double().numpy()
+    want = oracle.matmul_bt(W.bits(a), W.bits(b))
+    # bound from the arithmetic: the bf16 output is within half an ulp of the fp32 sum, and the
+    # fp32 sum of K products is within K * 2^-24 * sum_k |a_k b_k| of the exact one (generous:
+    # the tensor core's accumulation order is unspecified)
+    absab = np.abs(oracle.bf16_to_f64(W.bits(a))) @ np.abs(oracle.bf16_to_f64(W.bits(b))).T
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), 1e-30))) - 7)
+    bound = 0.5 * ulp * 2 + K * 2.0 ** -24 * absab + 1e-30
+    assert np.all(np.abs(got - want) <= bound), (M, N, K, float(np.max(np.abs(got - want) / bound)))
+    mx, mean = _rel_errors(got, want)
+    assert mx < 3e-2 and mean < 2e-3
+
+
+def test_lowrank_projection_wan_shape():
+    """V projection of the Wan layer through its rank-1413 (padded 1416) factors, 4680 tokens."""
+    d, M = W.MODEL_DIM, 4680
+    r = lowrank.retained_rank(d)
+    Wt = W.gen_weight(21, d, d)
+    w1, w2 = lowrank.svd_factors(Wt, r)
+    x = W.gen_act(22, M, d)
+    y = binding.lowrank_linear(x.cuda(), w1.cuda(), w2.cuda()).cpu().double().numpy()
+    want_t = oracle.lowrank_linear(W.bits(x), W.bits(w1), W.bits(w2), round_t=True)
+    mx, mean = _rel_errors(y, want_t)
+    assert mx < 2e-2 and mean < 3e-3, (mx, mean)
+    want = oracle.lowrank_linear(W.bits(x), W.bits(w1), W.bits(w2))
+    mx, mean = _rel_errors(y, want)
+    assert mx < 3e-2 and mean < 4e-3, (mx, mean)
+
+
+def test_full_rank_factors_reproduce_the_linear_layer():
+    d, M = 256, 300
+    Wt = W.gen_weight(5, d, d)
+    w1, w2 = lowrank.svd_factors(Wt, d)
+    x = W.gen_act(6, M, d)
+    y = binding.lowrank_linear(x.cuda(), w1.cuda(), w2.cuda()).cpu().double().numpy()
+    full = x.double().numpy() @ Wt.double().numpy().T
+    mx, mean = _rel_errors(y, full)
+    assert mx < 5e-2 and mean < 1e-2, (mx, mean)   # bf16 factors and intermediate
+
+
+def test_gemm_deterministic_and_no_device_error():
+    a = W.gen_act(1, 1000, 512).cuda()
+    b = W.gen_act(2, 768, 512).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c1 = binding.gemm_bf16(a, b, dev_error=err)
+    c2 = binding.gemm_bf16(a, b, dev_error=err)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2)
+    assert int(err.item()) == 0
