@@ -466,6 +466,63 @@ def run_lowrank(args, rank, local_rank, world):
         flush=True)
 
 
+def run_clip(args, rank, local_rank, world):
+    """The 5-s clip through 30 attention layers (Table 3 schedule: 23 forwards), eagerly and as
+    one CUDA graph; inputs of all 690 calls pre-generated on the device."""
+    import torch
+    from causal_video_diffusion_b200 import clip
+    from causal_video_diffusion_b200 import workloads as W
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS["clip30"]
+    drv = clip.ClipDriver(wl, seed=args.seed, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    drv.run()                                  # warm-up (first calls set kernel attributes)
+    torch.cuda.synchronize()
+    drv.reset()
+    e0, e1 = ev(), ev()
+    e0.record()
+    drv.run()
+    e1.record()
+    e1.synchronize()
+    eager_ms = e0.elapsed_time(e1)
+    drv.reset()
+    drv.capture()
+    for _ in range(max(1, args.warmup // 3)):
+        drv.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    reps = max(1, min(args.steps, 10))
+    e0, e1 = ev(), ev()
+    e0.record()
+    for _ in range(reps):
+        drv.replay()
+    e1.record()
+    e1.synchronize()
+    clocks = sampler.stop()
+    graph_ms = e0.elapsed_time(e1) / reps
+    for c in drv.caches:
+        if c.device_error() != 0:
+            raise RuntimeError("device error in the clip")
+    flops = drv.attn_flops()
+    peaks, src = load_peaks()
+    tf = flops / (graph_ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "attention-layer TFLOP/s over a 5-s clip (30 layers x 23 forwards)",
+        "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": reps,
+        "warmup": args.warmup, "ms_per_step": round(graph_ms, 3), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic seeded N(0,1) bf16 q/k/v per (forward, layer)",
+        "config": {"workload": "clip30: 7 chunks x (5,3,3,3,3,3,3) forwards x 30 layers, W=9",
+                   "calls": drv.calls, "graph": "one CUDA graph per clip"},
+        "eager_ms_per_clip": round(eager_ms, 3),
+        "chunk_steps_per_s": round(drv.calls / (graph_ms * 1e-3), 1),
+        "attention_only_frames_per_s": round(81 / (graph_ms * 1e-3), 1),
+        "gpu_launches": (2 * drv.layers + 1) * len(drv.sched),
+        "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "clocks": clocks}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -487,6 +544,8 @@ def main():
         run_reference(args, rank, world)
     elif args.workload == "lowrank_vo":
         run_lowrank(args, rank, local_rank, world)
+    elif args.workload == "clip30":
+        run_clip(args, rank, local_rank, world)
     else:
         run_ours(args, rank, local_rank, world)
 

@@ -80,6 +80,8 @@ _SIGNATURES = {
     "unstep_lowrank_linear": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "unstep_renoise": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong,
+                        ctypes.c_float, ctypes.c_void_p], ctypes.c_int),
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),
@@ -191,6 +193,12 @@ class LayerCache:
         self.device = dev
         with torch.cuda.device(dev):
             _check(L.unstep_cache_init(ctypes.byref(c), _stream_handle(stream)),
+                   "unstep_cache_init")
+
+    def reset(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Back to an empty cache (zeroed K/V, no frames), as after construction."""
+        with torch.cuda.device(self.device):
+            _check(lib().unstep_cache_init(ctypes.byref(self.c), _stream_handle(stream)),
                    "unstep_cache_init")
 
     # -- metadata ---------------------------------------------------------------------------
@@ -404,6 +412,20 @@ def lowrank_linear(x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                                        _dev_ptr(err, "dev_error"), _stream_handle(stream)),
            "unstep_lowrank_linear")
     return y
+
+
+def renoise(x0: torch.Tensor, eps: torch.Tensor, sigma: float,
+            out: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """out = (1 - sigma) * x0 + sigma * eps (bf16 latents of any shape)."""
+    if x0.dtype != torch.bfloat16 or eps.dtype != torch.bfloat16 or x0.shape != eps.shape:
+        raise ValueError("x0 and eps must be bf16 tensors of one shape")
+    if out is None:
+        out = torch.empty_like(x0)
+    _check(lib().unstep_renoise(_dev_ptr(x0, "x0"), _dev_ptr(eps, "eps"), _dev_ptr(out, "out"),
+                                x0.numel(), float(sigma), _stream_handle(stream)),
+           "unstep_renoise")
+    return out
 
 
 def selftest_wait_timeout(dev_error: torch.Tensor, limit_ns: int,

@@ -528,6 +528,20 @@ int unstep_lowrank_linear(const void *x, const void *w1, const void *w2, void *t
   return unstep_gemm_bf16(t, rank, w2, rank, y, d_out, M, d_out, rank, dev_error, stream);
 }
 
+int unstep_renoise(const void *x0, const void *eps, void *out, long long n, float sigma,
+                   unstep_stream_t stream) {
+  if (!x0 || !eps || !out || n < 0) return UNSTEP_ERR_ARG;
+  if (!(sigma >= 0.f && sigma <= 1.f)) return UNSTEP_ERR_ARG;
+  if (!aligned16(x0) || !aligned16(eps) || !aligned16(out)) return UNSTEP_ERR_ALIGN;
+  if (n == 0) return UNSTEP_OK;
+  if (unstep::launch_renoise(x0, eps, out, n, sigma, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
 int unstep_get_device_error(const unstep_cache_t *cache, unstep_stream_t stream) {
   if (!cache || !cache->dev_error) return UNSTEP_ERR_ARG;
   int v = 0;

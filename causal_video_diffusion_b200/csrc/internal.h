@@ -102,6 +102,10 @@ cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cuda
 cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
                                 int N, int K, int ldc, int *dev_error, cudaStream_t stream);
 
+// out[i] = (1 - sigma) * x0[i] + sigma * eps[i], bf16, n elements.
+cudaError_t launch_renoise(const void *x0, const void *eps, void *out, long long n, float sigma,
+                           cudaStream_t stream);
+
 // Size of the library's fixed device scratch buffer (see unstep_window_attn_noalloc).
 constexpr size_t kStaticScratchBytes = 48ull << 20;
 

@@ -235,6 +235,16 @@ int unstep_lowrank_linear(const void *x, const void *w1, const void *w2, void *t
                           int d_in, int rank, int d_out, int *dev_error, unstep_stream_t stream);
 
 /*
+ * Renoise (UnStep, abstract; Tables 4 and 5: the generated latent is renoised to the near-clean
+ * level sigma* = 0.02 before the clean-cache pass; a few-step student moves between its
+ * denoising steps the same way): out = (1 - sigma) * x0 + sigma * eps elementwise over n bf16
+ * values, in fp32 (one fma), rounded to bf16 (RNE).  out may alias x0 or eps.  0 <= sigma <= 1.
+ * Errors: ARG, ALIGN, CUDA.
+ */
+int unstep_renoise(const void *x0, const void *eps, void *out, long long n, float sigma,
+                   unstep_stream_t stream);
+
+/*
  * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported
  * an error); CUDA if the copy or the synchronisation itself failed.
  */

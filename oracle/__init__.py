@@ -343,3 +343,12 @@ def svd_truncate(W: np.ndarray, rank: int):
     (w1 = (V_r S_r)^T [rank][d_in], w2 = U_r [d_out][rank], singular values)."""
     U, S, Vh = np.linalg.svd(np.asarray(W, dtype=np.float64), full_matrices=False)
     return (S[:rank, None] * Vh[:rank]), U[:, :rank], S
+
+
+# --------------------------------------------------------------------------------------------
+# Renoise (abstract; Tables 4 and 5: renoise the generated latent to sigma* before the clean pass)
+# --------------------------------------------------------------------------------------------
+
+def renoise(x0_bits: np.ndarray, eps_bits: np.ndarray, sigma: float) -> np.ndarray:
+    """(1 - sigma) x0 + sigma eps in fp64 from bf16 bit patterns."""
+    return (1.0 - sigma) * bf16_to_f64(x0_bits) + sigma * bf16_to_f64(eps_bits)
