@@ -158,6 +158,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], int col0, int
                                           uint64_t sc2, uint64_t nm2, uint64_t (&acc)[4],
                                           uint32_t taddr) {
   uint32_t w[16];
+
 #pragma unroll
   for (int pi = 0; pi < 16; ++pi) {
     const uint64_t x2 = ffma2(f2_make(__uint_as_float(s[2 * pi]), __uint_as_float(s[2 * pi + 1])),
