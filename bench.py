@@ -81,10 +81,11 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, rope_q: bool = False):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"window_attn_{workload}.txt")
+    current kernel source (else None); ``rope_q``: the instantiation with the query prologue."""
+    name = f"window_attn_qrope_{workload}.txt" if rope_q else f"window_attn_{workload}.txt"
+    path = os.path.join(ROOT, "profiles", name)
     try:
         text = open(path).read()
     except OSError:
@@ -197,13 +198,16 @@ def run_ours(args, rank, local_rank, world):
     if cache.device_error() != 0:
         raise RuntimeError("device error during cache fill")
 
+    fq = args.q_rope == "attn"   # queries rotated inside the attention, not by the append
+
     def one_step(ev):
         q_work.copy_(q_src)
         flush_l2()                          # evict L2 between timed steps
         ev[0].record(stream)
-        cache.rope_kv_append(q_work, k_src, v_src, f_last, F)   # re-forward of the last chunk
+        # re-forward of the last chunk
+        cache.rope_kv_append(q_work, k_src, v_src, f_last, F, defer_q=fq)
         ev[1].record(stream)
-        cache.window_attn(q_work, wl.window, out=out)
+        cache.window_attn(q_work, wl.window, out=out, rope_q=fq)
         ev[2].record(stream)
 
     for _ in range(args.warmup):
@@ -239,7 +243,7 @@ def run_ours(args, rank, local_rank, world):
     k_h = k_src.cpu().pin_memory()
     v_h = v_src.cpu().pin_memory()
     out_h = torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16).pin_memory()
-    pipe = binding.HostStepPipeline(cache)
+    pipe = binding.HostStepPipeline(cache, rope_q_in_attn=fq)
     e2e_steps = max(4, min(args.steps, 100))
     pipe.run(q_h, k_h, v_h, f_last, F, wl.window, out_h, 4)            # warm-up
     e2e_ms = reduce_max(pipe.run(q_h, k_h, v_h, f_last, F, wl.window, out_h, e2e_steps)
@@ -251,7 +255,7 @@ def run_ours(args, rank, local_rank, world):
     attn_avg = reduce_max(sum(attn_ms) / args.steps, world, dev)
     rope_avg = reduce_max(sum(rope_ms) / args.steps, world, dev)
     attn_tflops = flops / (attn_avg * 1e-3) / 1e12
-    rope_bytes = wl.rope_bytes()
+    rope_bytes = wl.rope_bytes(rotate_q=not fq)
     rope_gbs = rope_bytes / (rope_avg * 1e-3) / 1e9
     value = world * flops / (step_ms * 1e-3) / 1e12
     act_bytes = s.B * s.L * s.H * s.D * 2
@@ -275,6 +279,8 @@ def run_ours(args, rank, local_rank, world):
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, then "
                   f"{L2_FLUSH_BYTES >> 20} MiB read)",
             "parallelism": f"independent streams x{world}",
+            "q_rope": "in the attention prologue (append moves k, v only)" if fq else
+                      "in the append (q rotated in place)",
         },
         "chunk_steps_per_s": round(world * s.B / (step_ms * 1e-3), 2),
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
@@ -286,7 +292,7 @@ def run_ours(args, rank, local_rank, world):
         "gpu_launches": 2 * args.steps,
         "gpu_launches_e2e": 2 * e2e_steps,
         "roofline": {
-            "kernel": f"window_attn_kernel<{s.D}>",
+            "kernel": f"window_attn_kernel<{s.D}, {str(fq).lower()}>",
             "bound": "tensor",
             "achieved": round(attn_tflops, 2),
             "peak": peaks["bf16_tflops"],
@@ -294,12 +300,12 @@ def run_ours(args, rank, local_rank, world):
             "unit": "TFLOP/s",
             "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
             "frac_of_sustained": round(attn_tflops / peaks["bf16_tflops_sustained"], 4),
-            "traffic": profiled_traffic(wl.name),
+            "traffic": profiled_traffic(wl.name, rope_q=fq),
             "ms_per_launch": round(attn_avg, 4),
             "flops_per_launch": flops,
         },
         "rope_roofline": {
-            "kernel": f"rope_kv_append_kernel<{s.D}>",
+            "kernel": f"rope_kv_append_kernel<{s.D}, {str(not fq).lower()}>",
             "bound": "hbm",
             "achieved": round(rope_gbs, 1),
             "peak": peaks["hbm_gbs"],
@@ -534,6 +540,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024, help="oracle rows per head (baseline)")
     ap.add_argument("--ref-rows", type=int, default=32, help="oracle rows per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--q-rope", choices=["append", "attn"], default="append",
+                    help="where the queries are rotated: in the append (q in place) or in the "
+                         "attention's prologue")
     args = ap.parse_args()
     rank, local_rank, world = dist_env()
     if world != args.gpus and "WORLD_SIZE" in os.environ:

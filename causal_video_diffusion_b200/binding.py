@@ -26,6 +26,9 @@ UNSTEP_ERR_CUDA = -7
 UNSTEP_ERR_DEVICE_TIMEOUT = -8
 UNSTEP_ERR_SCRATCH_LIMIT = -9
 
+UNSTEP_APPEND_DEFER_Q_ROPE = 1   # unstep_rope_kv_append_ex: leave q alone
+UNSTEP_ATTN_ROPE_Q = 1           # unstep_window_attn_ex: q is un-rotated, rotate it in-kernel
+
 
 class unstep_cache_t(ctypes.Structure):
     _fields_ = [
@@ -67,10 +70,15 @@ _SIGNATURES = {
     "unstep_rope_kv_append": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                ctypes.POINTER(unstep_cache_t), ctypes.c_int, unstep_grid_t,
                                ctypes.c_void_p], ctypes.c_int),
+    "unstep_rope_kv_append_ex": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.POINTER(unstep_cache_t), ctypes.c_int, unstep_grid_t,
+                                  ctypes.c_uint, ctypes.c_void_p], ctypes.c_int),
     "unstep_window_plan": ([ctypes.POINTER(unstep_cache_t), ctypes.c_int,
                             ctypes.POINTER(unstep_window_plan_t)], ctypes.c_int),
     "unstep_window_attn": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t), ctypes.c_int,
                             ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "unstep_window_attn_ex": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t), ctypes.c_int,
+                               ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p], ctypes.c_int),
     "unstep_window_attn_noalloc": ([ctypes.c_void_p, ctypes.POINTER(unstep_cache_t),
                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
                                    ctypes.c_int),
@@ -241,31 +249,56 @@ class LayerCache:
                "unstep_window_plan")
         return plan
 
-    def rope_kv_append(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+    def rope_kv_append(self, q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tensor,
                        frame_idx: int, frames: int,
-                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-        """Rotate q in place, append rotated k and v to the ring; returns q."""
+                       stream: Optional[torch.cuda.Stream] = None,
+                       defer_q: bool = False) -> Optional[torch.Tensor]:
+        """Rotate q in place, append rotated k and v to the ring; returns q.
+
+        ``defer_q``: q is left alone (it may be None) and only k, v are processed; the queries
+        are then rotated inside :meth:`window_attn` with ``rope_q=True``.
+        """
         L = self.chunk_len(frames)
-        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        acts = ((k, "k"), (v, "v")) if defer_q and q is None else ((q, "q"), (k, "k"), (v, "v"))
+        for t, n in acts:
             self._check_act(t, L, n)
         g = unstep_grid_t(frames, self.c.Hg, self.c.Wg)
-        rc = lib().unstep_rope_kv_append(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
-                                         ctypes.byref(self.c), int(frame_idx), g,
-                                         _stream_handle(stream))
-        _check(rc, "unstep_rope_kv_append")
+        qp = None if q is None else _dev_ptr(q, "q")
+        if defer_q:
+            rc = lib().unstep_rope_kv_append_ex(qp, _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                                ctypes.byref(self.c), int(frame_idx), g,
+                                                UNSTEP_APPEND_DEFER_Q_ROPE,
+                                                _stream_handle(stream))
+            _check(rc, "unstep_rope_kv_append_ex")
+        else:
+            rc = lib().unstep_rope_kv_append(qp, _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                             ctypes.byref(self.c), int(frame_idx), g,
+                                             _stream_handle(stream))
+            _check(rc, "unstep_rope_kv_append")
         return q
 
     def window_attn(self, q: torch.Tensor, window: int, out: Optional[torch.Tensor] = None,
-                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-        """Attention of the latest chunk's rotated queries over the last ``window`` frames."""
+                    stream: Optional[torch.cuda.Stream] = None,
+                    rope_q: bool = False) -> torch.Tensor:
+        """Attention of the latest chunk's queries over the last ``window`` frames.
+
+        q is the rotated queries (as :meth:`rope_kv_append` leaves them), or with ``rope_q`` the
+        un-rotated ones, which the kernel rotates after loading them.
+        """
         L = self.chunk_len(self.c.last_chunk_frames)
         self._check_act(q, L, "q")
         if out is None:
             out = torch.empty_like(q)
         self._check_act(out, L, "out")
-        rc = lib().unstep_window_attn(_dev_ptr(q, "q"), ctypes.byref(self.c), int(window),
-                                      _dev_ptr(out, "out"), _stream_handle(stream))
-        _check(rc, "unstep_window_attn")
+        if rope_q:
+            rc = lib().unstep_window_attn_ex(_dev_ptr(q, "q"), ctypes.byref(self.c), int(window),
+                                             _dev_ptr(out, "out"), UNSTEP_ATTN_ROPE_Q,
+                                             _stream_handle(stream))
+            _check(rc, "unstep_window_attn_ex")
+        else:
+            rc = lib().unstep_window_attn(_dev_ptr(q, "q"), ctypes.byref(self.c), int(window),
+                                          _dev_ptr(out, "out"), _stream_handle(stream))
+            _check(rc, "unstep_window_attn")
         return out
 
     def device_error(self, stream: Optional[torch.cuda.Stream] = None) -> int:
@@ -273,19 +306,22 @@ class LayerCache:
 
     def step_from_host(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor,
                        frame_idx: int, frames: int, window: int, out_h: torch.Tensor,
-                       bufs: dict, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                       bufs: dict, stream: Optional[torch.cuda.Stream] = None,
+                       rope_q_in_attn: bool = False) -> torch.Tensor:
         """One layer step from pinned host tensors: copy in, append, attend, copy out.
 
         ``bufs`` holds the device staging tensors ``q``, ``k``, ``v``, ``out`` (reused).
         The copies and both calls are enqueued on the stream; ``out_h`` is valid after a sync.
+        ``rope_q_in_attn``: deferred-q append, queries rotated inside the attention.
         """
         s = stream if stream is not None else torch.cuda.current_stream()
         with torch.cuda.stream(s):
             bufs["q"].copy_(q_h, non_blocking=True)
             bufs["k"].copy_(k_h, non_blocking=True)
             bufs["v"].copy_(v_h, non_blocking=True)
-            self.rope_kv_append(bufs["q"], bufs["k"], bufs["v"], frame_idx, frames, stream=s)
-            self.window_attn(bufs["q"], window, out=bufs["out"], stream=s)
+            self.rope_kv_append(bufs["q"], bufs["k"], bufs["v"], frame_idx, frames, stream=s,
+                                defer_q=rope_q_in_attn)
+            self.window_attn(bufs["q"], window, out=bufs["out"], stream=s, rope_q=rope_q_in_attn)
             out_h.copy_(bufs["out"], non_blocking=True)
         return out_h
 
@@ -300,10 +336,11 @@ class HostStepPipeline:
     across the host link.
     """
 
-    def __init__(self, cache: LayerCache, device=None):
+    def __init__(self, cache: LayerCache, device=None, rope_q_in_attn: bool = False):
         c = cache.c
         dev = cache.device if device is None else torch.device(device)
         self.cache = cache
+        self.rope_q_in_attn = rope_q_in_attn   # deferred-q append + in-kernel query RoPE
         self.h2d = torch.cuda.Stream(device=dev)
         self.d2h = torch.cuda.Stream(device=dev)
         self.compute = torch.cuda.Stream(device=dev)
@@ -346,9 +383,11 @@ class HostStepPipeline:
                 self.compute.wait_event(in_ready[b])
                 if out_done[b] is not None:
                     self.compute.wait_event(out_done[b])  # its output has left the device
+                fq = self.rope_q_in_attn
                 self.cache.rope_kv_append(bufs["q"], bufs["k"], bufs["v"], frame_idx, frames,
-                                          stream=self.compute)
-                self.cache.window_attn(bufs["q"], window, out=bufs["out"], stream=self.compute)
+                                          stream=self.compute, defer_q=fq)
+                self.cache.window_attn(bufs["q"], window, out=bufs["out"], stream=self.compute,
+                                       rope_q=fq)
                 computed[b] = ev()
                 computed[b].record(self.compute)
             with torch.cuda.stream(self.d2h):

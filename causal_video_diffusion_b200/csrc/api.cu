@@ -240,16 +240,20 @@ int unstep_append_plan(const unstep_cache_t *cache, int frame_idx, unstep_grid_t
   return is_new;
 }
 
-int unstep_rope_kv_append(void *q, const void *k, const void *v, unstep_cache_t *cache,
-                          int frame_idx, unstep_grid_t grid, unstep_stream_t stream) {
+int unstep_rope_kv_append_ex(void *q, const void *k, const void *v, unstep_cache_t *cache,
+                             int frame_idx, unstep_grid_t grid, unsigned flags,
+                             unstep_stream_t stream) {
   int rc = check_ready(cache);
   if (rc) return rc;
-  if (!q || !k || !v) return UNSTEP_ERR_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return UNSTEP_ERR_ALIGN;
+  if (flags & ~static_cast<unsigned>(UNSTEP_APPEND_DEFER_Q_ROPE)) return UNSTEP_ERR_ARG;
+  const bool rotate_q = !(flags & UNSTEP_APPEND_DEFER_Q_ROPE);
+  if ((rotate_q && !q) || !k || !v) return UNSTEP_ERR_ARG;
+  if ((rotate_q && !aligned16(q)) || !aligned16(k) || !aligned16(v)) return UNSTEP_ERR_ALIGN;
   const int is_new = unstep_append_plan(cache, frame_idx, grid, nullptr);
   if (is_new < 0) return is_new;
   unstep::RopeAppendParams p{};
-  p.q = q;
+  p.q = rotate_q ? q : nullptr;
+  p.rotate_q = rotate_q ? 1 : 0;
   p.k = k;
   p.v = v;
   p.k_cache = cache->k_cache;
@@ -286,6 +290,11 @@ int unstep_rope_kv_append(void *q, const void *k, const void *v, unstep_cache_t 
   return UNSTEP_OK;
 }
 
+int unstep_rope_kv_append(void *q, const void *k, const void *v, unstep_cache_t *cache,
+                          int frame_idx, unstep_grid_t grid, unstep_stream_t stream) {
+  return unstep_rope_kv_append_ex(q, k, v, cache, frame_idx, grid, 0u, stream);
+}
+
 int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_plan_t *plan) {
   int rc = check_shape(cache);
   if (rc) return rc;
@@ -315,10 +324,11 @@ int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_pl
   return UNSTEP_OK;
 }
 
-int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
-                       unstep_stream_t stream) {
+int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window, void *out,
+                          unsigned flags, unstep_stream_t stream) {
   int rc = check_ready(cache);
   if (rc) return rc;
+  if (flags & ~static_cast<unsigned>(UNSTEP_ATTN_ROPE_Q)) return UNSTEP_ERR_ARG;
   if (!q || !out) return UNSTEP_ERR_ARG;
   if (!aligned16(q) || !aligned16(out)) return UNSTEP_ERR_ALIGN;
   unstep_window_plan_t plan;
@@ -392,12 +402,39 @@ int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, v
   }
   p.scale_log2 = static_cast<float>(1.4426950408889634073599 / std::sqrt(static_cast<double>(D)));
   p.wait_limit_ns = unstep::kWaitLimitNs;
+  if (flags & UNSTEP_ATTN_ROPE_Q) {
+    // q is the latest chunk's un-rotated queries: row l is token (i, y, x) of frame
+    // last_chunk_start + i, rotated with the append's tables in the kernel's prologue
+    const float2 *tab = reinterpret_cast<const float2 *>(cache->cos_sin);
+    p.rope_q = 1;
+    p.tab_t = tab;
+    p.tab_h = p.tab_t + static_cast<size_t>(cache->max_pos_t) * (cache->d_t / 2);
+    p.tab_w = p.tab_h + static_cast<size_t>(cache->Hg) * (cache->d_h / 2);
+    p.half_t = cache->d_t / 2;
+    p.half_h = cache->d_h / 2;
+    p.half_w = cache->d_w / 2;
+    p.Tf = tf;
+    p.Wg = cache->Wg;
+    p.frame0 = cache->last_chunk_start;
+    p.frames = cache->last_chunk_frames;
+    const size_t tab_bytes = sizeof(float2) * (static_cast<size_t>(p.frames) * p.half_t +
+                                               static_cast<size_t>(cache->Hg) * p.half_h +
+                                               static_cast<size_t>(cache->Wg) * p.half_w);
+    p.tab_smem = tab_bytes <= static_cast<size_t>(unstep::kQRopeTabBytes) ? 1 : 0;
+    p.div_tf = unstep::make_fastdiv(static_cast<uint32_t>(tf));
+    p.div_wg = unstep::make_fastdiv(static_cast<uint32_t>(cache->Wg));
+  }
   if (unstep::launch_window_attn(D, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
   }
   return UNSTEP_OK;
+}
+
+int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
+                       unstep_stream_t stream) {
+  return unstep_window_attn_ex(q, cache, window, out, 0u, stream);
 }
 
 int unstep_window_attn_noalloc(const void *q, const unstep_cache_t *cache, int window,

@@ -28,6 +28,18 @@ inline FastDiv make_fastdiv(uint32_t d) {
 __device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv &f) {
   return (__umulhi(x, f.m) + x) >> f.l;
 }
+
+// One RoPE channel pair, two packed bf16 (a = low half, b = high half), rotated by (c, s):
+// (a c - b s, a s + b c) in fp32, each rounded to bf16 (RNE).  The append kernel and the
+// attention's query prologue both rotate through this function, so both give the same bits.
+__device__ __forceinline__ uint32_t rope_rotate_pair(uint32_t w, float2 cs) {
+  const float a = __uint_as_float(w << 16), b = __uint_as_float(w & 0xFFFF0000u);
+  const float ra = __fmaf_rn(a, cs.x, -__fmul_rn(b, cs.y));
+  const float rb = __fmaf_rn(a, cs.y, __fmul_rn(b, cs.x));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(rb), "f"(ra));
+  return r;
+}
 #endif
 
 struct RopeAppendParams {
@@ -46,6 +58,7 @@ struct RopeAppendParams {
   int frame_idx, frames, cap;
   int rows;       // cap * Tf
   int slot0;      // frame_idx mod cap
+  int rotate_q;   // 1: q rotated in place; 0: q neither read nor written
   FastDiv div_h;  // by H
   FastDiv div_l;  // by L
   FastDiv div_tf; // by Tf
@@ -81,7 +94,21 @@ struct AttnParams {
   unsigned epoch;    // 1 .. 2^24-1, distinct for consecutive launches
   FastDiv div_pairs; // by n_pairs
   FastDiv div_heads; // by H
+  // query RoPE in the prologue (rope_q != 0): q holds the chunk's un-rotated queries, chunk row
+  // l being token (i, y, x) of frame frame0 + i, l = i*Tf + y*Wg + x
+  int rope_q;
+  const float2 *tab_t, *tab_h, *tab_w;  // as in RopeAppendParams
+  int half_t, half_h, half_w;
+  int Tf, Wg, frame0, frames;
+  int tab_smem;      // 1: the chunk's rows fit in kQRopeTabBytes and are staged in shared memory
+  FastDiv div_tf;    // by Tf
+  FastDiv div_wg;    // by Wg
 };
+
+// Shared memory for the coefficient rows of the query rotation: frames*d_t/2 + Hg*d_h/2 +
+// Wg*d_w/2 float2 (14.3 KB for a 3-frame 30x52 chunk at 44/42/42); larger chunks read the
+// global tables instead.
+constexpr int kQRopeTabBytes = 24 * 1024;
 
 // Scratch layout shared by the host sizing and the kernel.
 constexpr size_t attn_counter_bytes(long long max_units) {

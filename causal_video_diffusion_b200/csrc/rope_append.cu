@@ -5,7 +5,9 @@
 // both in one pass over HBM: q, k, v are read once; rotated q goes back in place, rotated k and v
 // go to ring slot f mod cap.  The work is pure streaming (6 bf16 tensors of B*L*H*D elements),
 // so it is bound by HBM bandwidth: every thread moves 16-byte vectors, a warp covers 512
-// contiguous bytes of each input, and the coefficient tables (< 20 KB) stay in L1/L2.
+// contiguous bytes of each input, and the coefficient tables (< 20 KB) stay in L1/L2.  When the
+// attention rotates the queries itself (its query prologue), the K/V-only instantiation leaves q
+// alone and moves 4 of the 6 streams.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -17,7 +19,13 @@ constexpr int kThreads = 256;
 #ifndef UNSTEP_ROPE_ITEMS
 #define UNSTEP_ROPE_ITEMS 1
 #endif
-constexpr int kItemsPerThread = UNSTEP_ROPE_ITEMS;  // independent 16-byte vectors per thread
+// K/V-only form: two vectors of each of its two inputs per thread keep as many bytes in flight
+#ifndef UNSTEP_ROPE_ITEMS_KV
+#define UNSTEP_ROPE_ITEMS_KV 2
+#endif
+// independent 16-byte vectors (of each input) per thread
+template <bool kQ>
+constexpr int items_per_thread() { return kQ ? UNSTEP_ROPE_ITEMS : UNSTEP_ROPE_ITEMS_KV; }
 
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
   uint4 r;
@@ -29,22 +37,6 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
 
 __device__ __forceinline__ uint4 ld_plain(const void *p) {
   return *reinterpret_cast<const uint4 *>(p);
-}
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t pack_rn(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
-  return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// Rotate one packed bf16 pair (a = low, b = high) by (c, s): (a c - b s, a s + b c).
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float2 cs) {
-  const float a = bf_lo(w), b = bf_hi(w);
-  const float ra = fmaf(a, cs.x, -b * cs.y);
-  const float rb = fmaf(a, cs.y, b * cs.x);
-  return pack_rn(ra, rb);
 }
 
 struct Item {
@@ -89,9 +81,11 @@ __device__ __forceinline__ void locate(const RopeAppendParams &p, uint32_t it, I
   }
 }
 
-template <int D>
+// kQ: q is rotated in place; without it q is neither read nor written.
+template <int D, bool kQ>
 __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppendParams p,
                                                                    uint32_t n_items) {
+  constexpr int kItemsPerThread = items_per_thread<kQ>();
   const uint32_t base = blockIdx.x * (kThreads * kItemsPerThread) + threadIdx.x;
   if (blockIdx.x == 0 && threadIdx.x < p.frames) {
     const int f = p.frame_idx + threadIdx.x;
@@ -106,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
     live[u] = it < n_items;
     if (live[u]) {
       locate<D>(p, it, m[u]);
-      qv[u] = ld_plain(static_cast<const __nv_bfloat16 *>(p.q) + m[u].e);
+      if (kQ) qv[u] = ld_plain(static_cast<const __nv_bfloat16 *>(p.q) + m[u].e);
       kv[u] = ld_stream(static_cast<const __nv_bfloat16 *>(p.k) + m[u].e);
       vv[u] = ld_stream(static_cast<const __nv_bfloat16 *>(p.v) + m[u].e);
     }
@@ -114,16 +108,19 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
 #pragma unroll
   for (int u = 0; u < kItemsPerThread; ++u) {
     if (!live[u]) continue;
-    uint4 qo, ko;
-    qo.x = rotate_pair(qv[u].x, m[u].cs[0]);
-    qo.y = rotate_pair(qv[u].y, m[u].cs[1]);
-    qo.z = rotate_pair(qv[u].z, m[u].cs[2]);
-    qo.w = rotate_pair(qv[u].w, m[u].cs[3]);
-    ko.x = rotate_pair(kv[u].x, m[u].cs[0]);
-    ko.y = rotate_pair(kv[u].y, m[u].cs[1]);
-    ko.z = rotate_pair(kv[u].z, m[u].cs[2]);
-    ko.w = rotate_pair(kv[u].w, m[u].cs[3]);
-    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.q) + m[u].e) = qo;
+    if (kQ) {
+      uint4 qo;
+      qo.x = rope_rotate_pair(qv[u].x, m[u].cs[0]);
+      qo.y = rope_rotate_pair(qv[u].y, m[u].cs[1]);
+      qo.z = rope_rotate_pair(qv[u].z, m[u].cs[2]);
+      qo.w = rope_rotate_pair(qv[u].w, m[u].cs[3]);
+      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.q) + m[u].e) = qo;
+    }
+    uint4 ko;
+    ko.x = rope_rotate_pair(kv[u].x, m[u].cs[0]);
+    ko.y = rope_rotate_pair(kv[u].y, m[u].cs[1]);
+    ko.z = rope_rotate_pair(kv[u].z, m[u].cs[2]);
+    ko.w = rope_rotate_pair(kv[u].w, m[u].cs[3]);
     *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.k_cache) + m[u].ce) = ko;
     *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.v_cache) + m[u].ce) = vv[u];
   }
@@ -133,21 +130,27 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
 
 cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream) {
   const long long n_items = static_cast<long long>(p.B) * p.L * p.H * (p.D / 8);
-  if (n_items >= (1ll << 31) - kThreads * kItemsPerThread) return cudaErrorInvalidConfiguration;
+  const int items = p.rotate_q ? items_per_thread<true>() : items_per_thread<false>();
+  if (n_items >= (1ll << 31) - kThreads * items) return cudaErrorInvalidConfiguration;
   RopeAppendParams q = p;
   q.slot0 = p.frame_idx % p.cap;
   q.div_h = make_fastdiv(static_cast<uint32_t>(p.H));
   q.div_l = make_fastdiv(static_cast<uint32_t>(p.L));
   q.div_tf = make_fastdiv(static_cast<uint32_t>(p.Tf));
   q.div_wg = make_fastdiv(static_cast<uint32_t>(p.Wg));
-  const long long per_block = kThreads * kItemsPerThread;
+  const long long per_block = kThreads * items;
   long long blocks = (n_items + per_block - 1) / per_block;
   if (blocks < 1) blocks = 1;
   const uint32_t n = static_cast<uint32_t>(n_items);
-  if (p.D == 128) {
-    rope_kv_append_kernel<128><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(q, n);
+  const dim3 gb(static_cast<unsigned>(blocks));
+  if (p.D == 128 && p.rotate_q) {
+    rope_kv_append_kernel<128, true><<<gb, kThreads, 0, stream>>>(q, n);
+  } else if (p.D == 128) {
+    rope_kv_append_kernel<128, false><<<gb, kThreads, 0, stream>>>(q, n);
+  } else if (p.D == 64 && p.rotate_q) {
+    rope_kv_append_kernel<64, true><<<gb, kThreads, 0, stream>>>(q, n);
   } else if (p.D == 64) {
-    rope_kv_append_kernel<64><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(q, n);
+    rope_kv_append_kernel<64, false><<<gb, kThreads, 0, stream>>>(q, n);
   } else {
     return cudaErrorInvalidValue;
   }

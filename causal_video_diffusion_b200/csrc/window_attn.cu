@@ -17,6 +17,9 @@
 //   warp  9    MMA issuer (one thread): QK^T and PV for both tiles, ping-ponging so that the
 //              tensor core works on one tile while the other tile's softmax runs
 //   warps 10-11 idle (they complete the third warpgroup, whose registers the softmax takes)
+// When q arrives un-rotated, each softmax warpgroup first applies the 3D RoPE to its loaded Q
+// tile in shared memory (once per segment, from coefficient rows staged in shared memory),
+// before the MMA issuer may use it.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 //
 // The ring cache holds the window as at most two contiguous row ranges; each range is tiled on
@@ -59,7 +62,7 @@ constexpr uint64_t kDrainLimitNs = 1000000000ull;
 #define UNSTEP_KV_STAGES 4
 #endif
 
-template <int D>
+template <int D, bool kRopeQ = false>
 struct Cfg {
   static constexpr int kBoxes = D / 64;                // 128-byte swizzle boxes per row
   static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16
@@ -67,7 +70,8 @@ struct Cfg {
   static constexpr int kSmemQ = 0;
   static constexpr int kSmemKV = 2 * kTileBytes;
   static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
-  static constexpr int kSmemUsed = kSmemBar + 256;
+  static constexpr int kSmemTab = kSmemBar + 256;      // RoPE rows of the chunk (kRopeQ)
+  static constexpr int kSmemUsed = kSmemTab + (kRopeQ ? kQRopeTabBytes : 0);
   // at least ~116 KB so that a second CTA (which would block on TMEM) never shares the SM
   static constexpr int kSmemAlloc = (kSmemUsed + 1024 > 118 * 1024) ? kSmemUsed + 1024
                                                                     : 118 * 1024;
@@ -257,6 +261,94 @@ __device__ __forceinline__ UnitPos unit_pos(const AttnParams &p, int u) {
   return x;
 }
 
+// Coefficient rows the query rotation reads: the chunk's temporal rows (frames frame0 ..) and
+// the h and w tables, either staged in shared memory (t row i = frame frame0 + i) or in global
+// memory (t row = absolute frame).
+struct QTabs {
+  const float2 *t, *h, *w;
+  int t_base;  // added to the chunk-relative frame i
+};
+
+// Rotation of one query tile in shared memory (kRopeQ): the warpgroup's warp wq takes rows
+// wq, wq + 4, ...; a row is D channels in D/64 boxes of 128 bytes (128-byte swizzle: 16-byte
+// chunk c of row r sits at chunk c ^ (r mod 8)), and lane ln takes channels
+// [ln*D/32, (ln+1)*D/32), i.e. D/64 channel pairs, so that a warp's coefficient reads are one
+// contiguous run per axis block and its shared-memory accesses are conflict-free.  Rows past the
+// chunk end (TMA zero fill) are left as loaded.  The arithmetic is the append kernel's, so the
+// tile holds exactly what unstep_rope_kv_append would have written to q.
+template <int D>
+__device__ __forceinline__ void rope_q_tile(const AttnParams &p, const QTabs &tabs,
+                                            uint8_t *tile, int l0, int wq, int lane) {
+  constexpr int kPairs = D / 64;              // channel pairs per lane
+  const int ch0 = lane * (D / 32);            // first channel of the lane
+  const int box = ch0 >> 6;
+  const int byte_in_box = (ch0 & 63) * 2;
+  const int chunk = byte_in_box >> 4, sub = byte_in_box & 15;
+  const float2 *tb[kPairs];
+  int stride[kPairs], axis[kPairs];
+#pragma unroll
+  for (int u = 0; u < kPairs; ++u) {
+    const int pr = ch0 / 2 + u;
+    if (pr < p.half_t) {
+      axis[u] = 0;
+      tb[u] = tabs.t + pr;
+      stride[u] = p.half_t;
+    } else if (pr < p.half_t + p.half_h) {
+      axis[u] = 1;
+      tb[u] = tabs.h + (pr - p.half_t);
+      stride[u] = p.half_h;
+    } else {
+      axis[u] = 2;
+      tb[u] = tabs.w + (pr - p.half_t - p.half_h);
+      stride[u] = p.half_w;
+    }
+  }
+  // 32 rows per warp in batches of kBatch: every load of a batch is issued before its first
+  // use; rows past the chunk end decode a clamped position and skip only their store
+  constexpr int kBatch = 8;
+  const int n_live = min(128, p.L - l0);
+#pragma unroll 1
+  for (int r0 = 0; r0 < 128; r0 += 4 * kBatch) {
+    float2 cs[kBatch][kPairs];
+    uint32_t v[kBatch][kPairs];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int r = r0 + 4 * b + wq;
+      const uint32_t l = static_cast<uint32_t>(l0 + min(r, n_live - 1));
+      const uint32_t i = fdiv(l, p.div_tf);
+      const uint32_t tok = l - i * static_cast<uint32_t>(p.Tf);
+      const uint32_t y = fdiv(tok, p.div_wg);
+      const uint32_t x = tok - y * static_cast<uint32_t>(p.Wg);
+#pragma unroll
+      for (int u = 0; u < kPairs; ++u) {
+        const int pos = axis[u] == 0 ? static_cast<int>(i) + tabs.t_base
+                                     : (axis[u] == 1 ? static_cast<int>(y) : static_cast<int>(x));
+        cs[b][u] = tb[u][pos * stride[u]];
+      }
+      const uint8_t *a = tile + box * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4) + sub;
+      if constexpr (kPairs == 2) {
+        const uint2 w2 = *reinterpret_cast<const uint2 *>(a);
+        v[b][0] = w2.x;
+        v[b][kPairs - 1] = w2.y;
+      } else {
+        v[b][0] = *reinterpret_cast<const uint32_t *>(a);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int r = r0 + 4 * b + wq;
+      if (r >= n_live) continue;
+      uint8_t *a = tile + box * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4) + sub;
+      if constexpr (kPairs == 2) {
+        *reinterpret_cast<uint2 *>(a) = make_uint2(rope_rotate_pair(v[b][0], cs[b][0]),
+                                                   rope_rotate_pair(v[b][1], cs[b][1]));
+      } else {
+        *reinterpret_cast<uint32_t *>(a) = rope_rotate_pair(v[b][0], cs[b][0]);
+      }
+    }
+  }
+}
+
 // Named barrier of one softmax warpgroup (ids 1 and 2; 0 is __syncthreads).
 __device__ __forceinline__ void wg_sync(int i) {
   asm volatile("bar.sync %0, 128;" ::"r"(1 + i) : "memory");
@@ -360,12 +452,13 @@ UNSTEP_COLD_FN void merge_row(const AttnParams &p, int i, int row, long long t0,
   }
 }
 
-template <int D>
+// kRopeQ: q is un-rotated and the query prologue rotates it (warps 10 and 11).
+template <int D, bool kRopeQ>
 __global__ void __launch_bounds__(kThreads, 1)
     window_attn_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kRopeQ>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -379,7 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *p_ready = s_full + 2;
   uint64_t *o_done = p_ready + 2;
   uint64_t *drain = o_done + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *q_rot = drain + 1;    // query tiles rotated by both warpgroups (kRopeQ)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_rot + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *merge_word = reinterpret_cast<volatile int *>(tmem_slot + 2);  // [2]
 
@@ -400,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(q_rot, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -505,7 +600,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; ok && get_seg(p, cta, sk, q, sg); ++q) {
           const bool has1 = unit_pos(p, sg.u).has1;
           const int ntl = sg.k1 - sg.k0;
-          if (!(ok = wait_bounded(q_full, static_cast<uint32_t>(q) & 1u, g, E))) break;
+          if (!(ok = wait_bounded(kRopeQ ? q_rot : q_full, static_cast<uint32_t>(q) & 1u, g, E)))
+            break;
           if (!(ok = wait_full(n))) break;
           tc_fence_after();
           qk(0, n % NS);
@@ -569,11 +665,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kTileFloats = D * 128 + 256;  // one query tile of a scratch slot
     uint32_t cnt = 0;                           // key tiles this warpgroup has processed
     bool ok = true;
+    QTabs qt{p.tab_t, p.tab_h, p.tab_w, p.frame0};
+    if constexpr (kRopeQ) {
+      if (p.tab_smem) {
+        // the chunk's coefficient rows into shared memory, once per CTA, by both warpgroups
+        float2 *st = reinterpret_cast<float2 *>(smem + C::kSmemTab);
+        const int nt = p.frames * p.half_t, nh = (p.Tf / p.Wg) * p.half_h, nw = p.Wg * p.half_w;
+        const float2 *gt = p.tab_t + static_cast<long long>(p.frame0) * p.half_t;
+        // all of a thread's loads are issued before its stores (first touch: HBM latency once)
+        constexpr int kPer = kQRopeTabBytes / 8 / 256;
+        float2 tv[kPer];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+          const int e = threadIdx.x + 256 * k;
+          if (e < nt + nh + nw)
+            tv[k] = e < nt ? gt[e] : (e < nt + nh ? p.tab_h[e - nt] : p.tab_w[e - nt - nh]);
+        }
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+          const int e = threadIdx.x + 256 * k;
+          if (e < nt + nh + nw) st[e] = tv[k];
+        }
+        qt = QTabs{st, st + nt, st + nt + nh, 0};
+        asm volatile("bar.sync 3, 256;" ::: "memory");
+      }
+    }
     Seg sg;
     // Every segment is walked even after an abort (the work is skipped), so that the named
     // barriers of the warpgroup are always reached by all of its threads.
     for (int q = 0; get_seg(p, cta, sk, q, sg); ++q) {
       const UnitPos up = unit_pos(p, sg.u);
+      if constexpr (kRopeQ) {
+        // every segment's query tiles pass through both warpgroups before the MMA issuer may
+        // read them; warpgroup 1 takes part even when the segment has no second tile, so that
+        // every waiter on q_full observes its phases one by one
+        if (ok) ok = __all_sync(kFull, wait_bounded(q_full, static_cast<uint32_t>(q) & 1u, g, E));
+        if (ok && (i == 0 || up.has1))
+          rope_q_tile<D>(p, qt, smem + C::kSmemQ + i * C::kTileBytes, up.q0 + i * 128, wq, lane);
+        fence_proxy_async_smem();
+        mbar_arrive(q_rot);
+      }
       if (i == 1 && !up.has1) continue;
       const int ntl = sg.k1 - sg.k0;
       float m_run = -INFINITY, l_run = 0.f;
@@ -766,10 +897,10 @@ __global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_muf
   }
 }
 
-template <int D>
+template <int D, bool kRopeQ>
 cudaError_t launch_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      const AttnParams &p, cudaStream_t stream) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kRopeQ>;
   // the shared-memory opt-in is per device; remember which devices have it
   static unsigned long long attr_set = 0;
   int dev = 0;
@@ -777,14 +908,14 @@ cudaError_t launch_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (dev >= 64 || !(__atomic_load_n(&attr_set, __ATOMIC_ACQUIRE) & bit)) {
-    e = cudaFuncSetAttribute(window_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemAlloc);
+    e = cudaFuncSetAttribute(window_attn_kernel<D, kRopeQ>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) return e;
     if (dev < 64) __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
   if (p.grid < 1) return cudaErrorInvalidConfiguration;
-  window_attn_kernel<D><<<static_cast<unsigned>(p.grid), kThreads, C::kSmemAlloc, stream>>>(
-      tq, tk, tv, p);
+  window_attn_kernel<D, kRopeQ>
+      <<<static_cast<unsigned>(p.grid), kThreads, C::kSmemAlloc, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -793,8 +924,12 @@ cudaError_t launch_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
 cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
                                const CUtensorMap &tmap_v, const AttnParams &p,
                                cudaStream_t stream) {
-  if (D == 128) return launch_d<128>(tmap_q, tmap_k, tmap_v, p, stream);
-  if (D == 64) return launch_d<64>(tmap_q, tmap_k, tmap_v, p, stream);
+  if (D == 128)
+    return p.rope_q ? launch_d<128, true>(tmap_q, tmap_k, tmap_v, p, stream)
+                    : launch_d<128, false>(tmap_q, tmap_k, tmap_v, p, stream);
+  if (D == 64)
+    return p.rope_q ? launch_d<64, true>(tmap_q, tmap_k, tmap_v, p, stream)
+                    : launch_d<64, false>(tmap_q, tmap_k, tmap_v, p, stream);
   return cudaErrorInvalidValue;
 }
 

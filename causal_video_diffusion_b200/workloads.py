@@ -79,10 +79,11 @@ class Workload:
         s = self.shape
         return 4 * s.B * s.H * s.L * self.keys_for_chunk(chunk) * s.D
 
-    def rope_bytes(self) -> int:
-        """Algorithmic bytes of one RoPE+append call: read q, k, v; write q, K, V (bf16)."""
+    def rope_bytes(self, rotate_q: bool = True) -> int:
+        """Algorithmic bytes of one RoPE+append call: read q, k, v; write q, K, V (bf16).
+        Without ``rotate_q`` (queries rotated inside the attention): read k, v; write K, V."""
         s = self.shape
-        return 6 * s.B * s.L * s.H * s.D * 2
+        return (6 if rotate_q else 4) * s.B * s.L * s.H * s.D * 2
 
 
 WAN = dict(H=12, D=128, Hg=30, Wg=52, d_t=44, d_h=42, d_w=42)

@@ -167,6 +167,27 @@ int unstep_rope_kv_append(void *q, const void *k, const void *v, unstep_cache_t 
                           int frame_idx, unstep_grid_t grid, unstep_stream_t stream);
 
 /*
+ * Flags of unstep_rope_kv_append_ex.
+ *   UNSTEP_APPEND_DEFER_Q_ROPE: q is neither read nor written (it may be NULL); only k and v
+ *   are processed (4 of the 6 HBM streams).  The chunk's queries are then rotated by
+ *   unstep_window_attn_ex with UNSTEP_ATTN_ROPE_Q, inside the attention.
+ */
+#define UNSTEP_APPEND_DEFER_Q_ROPE 1u
+
+/*
+ * unstep_rope_kv_append with flags (0 = exactly unstep_rope_kv_append).
+ * Source: the paper's abstract (RoPE from cached coefficients, KV-cache indexing); applying the
+ * query half of the RoPE inside the attention call instead of in the append is this library's
+ * own fusion, which saves the round trip of q through HBM.  With UNSTEP_APPEND_DEFER_Q_ROPE the
+ * cache, slot_frame and metadata are updated exactly as without it, bit for bit, and q is
+ * untouched.
+ * Errors: those of unstep_rope_kv_append, plus ARG for an unknown flag bit.
+ */
+int unstep_rope_kv_append_ex(void *q, const void *k, const void *v, unstep_cache_t *cache,
+                             int frame_idx, unstep_grid_t grid, unsigned flags,
+                             unstep_stream_t stream);
+
+/*
  * Host-only window resolution for the latest chunk: the frames
  * [max(first_frame, f_end - window + 1), f_end], f_end the latest chunk's last frame, as at
  * most two contiguous row ranges of the ring.  Errors: ARG, WINDOW (no chunk appended yet, or
@@ -187,6 +208,26 @@ int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_pl
  */
 int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
                        unstep_stream_t stream);
+
+/*
+ * Flags of unstep_window_attn_ex.
+ *   UNSTEP_ATTN_ROPE_Q: q holds the latest chunk's UN-rotated queries (as produced by the
+ *   projection); the kernel rotates each query tile after loading it, with the cache's tables and
+ *   the positions of the latest appended chunk (frame last_chunk_start + i, grid y, x), exactly
+ *   as unstep_rope_kv_append would have rotated it.  q itself is not modified.
+ */
+#define UNSTEP_ATTN_ROPE_Q 1u
+
+/*
+ * unstep_window_attn with flags (0 = exactly unstep_window_attn).
+ * With UNSTEP_ATTN_ROPE_Q, the output is bit-identical to unstep_rope_kv_append (q rotated in
+ * place) followed by unstep_window_attn on that rotated q, for the same inputs.  Use it after
+ * unstep_rope_kv_append_ex with UNSTEP_APPEND_DEFER_Q_ROPE (or after a plain append whose q
+ * buffer was a copy).  The query rotation is done by two otherwise idle warps of each CTA.
+ * Errors: those of unstep_window_attn, plus ARG for an unknown flag bit.
+ */
+int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window, void *out,
+                          unsigned flags, unstep_stream_t stream);
 
 /*
  * unstep_window_attn for callers that cannot allocate device memory.

@@ -212,3 +212,44 @@ def test_multiply_high_division_method():
         hi = (xs_d.astype(object) * m) >> 32
         q = np.array([(int(h) + int(x)) >> l for h, x in zip(hi, xs_d)], dtype=np.int64)
         assert np.array_equal(q, xs_d // d), d
+
+
+def test_ex_entry_points_flags_and_errors(L):
+    """The flag forms of the append and the attention reject unknown flags; a deferred-q append
+    ignores q (NULL or misaligned); every failing call returns before any launch."""
+    s = W.WORKLOADS["tiny"].shape
+    c = _cache(s, 6, fake_ptrs=True)
+    c.initialized = INIT_MAGIC
+    c.frames_written, c.first_frame, c.last_chunk_start, c.last_chunk_frames = 6, 0, 3, 3
+    g = B.unstep_grid_t(3, 4, 6)
+    q = ctypes.c_void_p(0x600000)
+    odd = ctypes.c_void_p(0x600004)
+    defer = B.UNSTEP_APPEND_DEFER_Q_ROPE
+    assert L.unstep_rope_kv_append_ex(q, q, q, ctypes.byref(c), 6, g, 2, None) == B.UNSTEP_ERR_ARG
+    assert L.unstep_rope_kv_append_ex(q, q, q, ctypes.byref(c), 6, g, 0x80000000, None) == \
+        B.UNSTEP_ERR_ARG
+    # with the flag, q plays no part: NULL or misaligned q reach the frame-order check
+    assert L.unstep_rope_kv_append_ex(None, q, q, ctypes.byref(c), 0, g, defer, None) == \
+        B.UNSTEP_ERR_FRAME_ORDER
+    assert L.unstep_rope_kv_append_ex(odd, q, q, ctypes.byref(c), 0, g, defer, None) == \
+        B.UNSTEP_ERR_FRAME_ORDER
+    # without it q is checked first
+    assert L.unstep_rope_kv_append_ex(None, q, q, ctypes.byref(c), 0, g, 0, None) == \
+        B.UNSTEP_ERR_ARG
+    assert L.unstep_rope_kv_append_ex(odd, q, q, ctypes.byref(c), 0, g, 0, None) == \
+        B.UNSTEP_ERR_ALIGN
+    # k and v are still required
+    assert L.unstep_rope_kv_append_ex(None, None, q, ctypes.byref(c), 6, g, defer, None) == \
+        B.UNSTEP_ERR_ARG
+    assert L.unstep_rope_kv_append_ex(None, q, odd, ctypes.byref(c), 6, g, defer, None) == \
+        B.UNSTEP_ERR_ALIGN
+    rq = B.UNSTEP_ATTN_ROPE_Q
+    assert L.unstep_window_attn_ex(q, ctypes.byref(c), 6, q, 4, None) == B.UNSTEP_ERR_ARG
+    assert L.unstep_window_attn_ex(q, ctypes.byref(c), 7, q, rq, None) == B.UNSTEP_ERR_WINDOW
+    assert L.unstep_window_attn_ex(None, ctypes.byref(c), 6, q, rq, None) == B.UNSTEP_ERR_ARG
+    assert L.unstep_window_attn_ex(odd, ctypes.byref(c), 6, q, rq, None) == B.UNSTEP_ERR_ALIGN
+    c2 = _cache(s, 6, fake_ptrs=True)           # never initialised
+    assert L.unstep_window_attn_ex(q, ctypes.byref(c2), 6, q, rq, None) == B.UNSTEP_ERR_ARG
+    assert L.unstep_rope_kv_append_ex(None, q, q, ctypes.byref(c2), 0, g, defer, None) == \
+        B.UNSTEP_ERR_ARG
+    assert (c.frames_written, c.last_chunk_start, c.last_chunk_frames) == (6, 3, 3)
