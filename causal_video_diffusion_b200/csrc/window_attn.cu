@@ -108,35 +108,6 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
 #endif
 constexpr int kEmuPairsPer8 = UNSTEP_EMU_PAIRS_PER8;
 
-// Softmax in two passes over the scores in TMEM (max, then exponentials), so that only two
-// 32-column chunks of a row are in registers at a time, instead of one pass holding all 128.
-// Off by default: on B200 the extra TMEM reads and their exposed latency cost more than the
-// register relief gains (0.965 ms against 0.858 ms at the full-cache shape).
-#ifndef UNSTEP_SOFTMAX_TWO_PASS
-#define UNSTEP_SOFTMAX_TWO_PASS 0
-#endif
-
-// Max of one 32-column chunk (columns col0..col0+31; with `masked`, columns >= valid ignored):
-// independent 3-input max chains, then a short tree.
-__device__ __forceinline__ float chunk_max(const uint32_t (&s)[32], int col0, int valid,
-                                           bool masked) {
-  float v[32];
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    v[e] = __uint_as_float(s[e]);
-    if (masked && col0 + e >= valid) v[e] = -INFINITY;
-  }
-  float m4[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float m = fmax3(v[8 * k], v[8 * k + 1], v[8 * k + 2]);
-    m = fmax3(m, v[8 * k + 3], v[8 * k + 4]);
-    m = fmax3(m, v[8 * k + 5], v[8 * k + 6]);
-    m4[k] = fmaxf(m, v[8 * k + 7]);
-  }
-  return fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-}
-
 // Max of a row's 128 scores: eight independent chains of 3-input max, then a short tree.
 __device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
   float m8[8];
@@ -409,50 +380,59 @@ __device__ __forceinline__ int piece_slot(const AttnParams &p, int c, long long 
 }
 
 // Merge the pieces of CTAs c_first..c_last for one row: rescale each to the common max,
-// sum, normalise, store.
+// sum, normalise, store.  The merge only reads L2 and is bound by its latency: each step takes
+// one piece's max and kMergeCB of its channels in one round trip, so the number of round trips
+// is (D / kMergeCB) x pieces.  Piece c > c_first is the first piece of its CTA (slot 2c): its
+// range starts inside the unit; only c_first's slot needs the range test.
+#ifndef UNSTEP_MERGE_CB
+#define UNSTEP_MERGE_CB 32
+#endif
 template <int D>
 UNSTEP_COLD_FN void merge_row(const AttnParams &p, int i, int row, long long t0,
-                                       int c_first, int c_last, __nv_bfloat16 *dst, bool live) {
+                              int c_first, int c_last, __nv_bfloat16 *dst, bool live) {
   constexpr int kTileFloats = D * 128 + 256;
+  constexpr int kCB = UNSTEP_MERGE_CB;
   __threadfence();
+  const int first_slot = piece_slot(p, c_first, t0);
+  auto piece = [&](int c) {
+    return p.slots + static_cast<long long>(c == c_first ? first_slot : 2 * c) * p.slot_floats +
+           i * kTileFloats + row;
+  };
   float M = -INFINITY;
 #pragma unroll 1
-  for (int c = c_first; c <= c_last; ++c) {
-    const float *src =
-        p.slots + static_cast<long long>(piece_slot(p, c, t0)) * p.slot_floats + i * kTileFloats;
-    M = fmaxf(M, __ldcg(src + D * 128 + row));
-  }
+  for (int c = c_first; c <= c_last; ++c) M = fmaxf(M, __ldcg(piece(c) + D * 128));
   float Lsum = 0.f;
 #pragma unroll 1
   for (int c = c_first; c <= c_last; ++c) {
-    const float *src =
-        p.slots + static_cast<long long>(piece_slot(p, c, t0)) * p.slot_floats + i * kTileFloats;
-    Lsum += __ldcg(src + D * 128 + 128 + row) * ex2_approx(__ldcg(src + D * 128 + row) - M);
+    const float *src = piece(c);
+    Lsum += __ldcg(src + D * 128 + 128) * ex2_approx(__ldcg(src + D * 128) - M);
   }
   const float inv = 1.f / Lsum;
 #pragma unroll 1
-  for (int c8 = 0; c8 < D / 8; ++c8) {
-    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int cb = 0; cb < D / kCB; ++cb) {
+    float a[kCB];
+#pragma unroll
+    for (int e = 0; e < kCB; ++e) a[e] = 0.f;
 #pragma unroll 1
     for (int c = c_first; c <= c_last; ++c) {
-      const float *src =
-          p.slots + static_cast<long long>(piece_slot(p, c, t0)) * p.slot_floats + i * kTileFloats;
-      const float w = ex2_approx(__ldcg(src + D * 128 + row) - M);
+      const float *src = piece(c);
+      const float w = ex2_approx(__ldcg(src + D * 128) - M);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a[e] = fmaf(w, __ldcg(src + (c8 * 8 + e) * 128 + row), a[e]);
+      for (int e = 0; e < kCB; ++e) a[e] = fmaf(w, __ldcg(src + (cb * kCB + e) * 128), a[e]);
     }
     if (live) {
-      uint4 v;
-      v.x = pack_bf16x2(a[0] * inv, a[1] * inv);
-      v.y = pack_bf16x2(a[2] * inv, a[3] * inv);
-      v.z = pack_bf16x2(a[4] * inv, a[5] * inv);
-      v.w = pack_bf16x2(a[6] * inv, a[7] * inv);
-      *reinterpret_cast<uint4 *>(dst + c8 * 8) = v;
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst + cb * kCB);
+#pragma unroll
+      for (int q = 0; q < kCB / 8; ++q)
+        d4[q] = make_uint4(pack_bf16x2(a[8 * q] * inv, a[8 * q + 1] * inv),
+                           pack_bf16x2(a[8 * q + 2] * inv, a[8 * q + 3] * inv),
+                           pack_bf16x2(a[8 * q + 4] * inv, a[8 * q + 5] * inv),
+                           pack_bf16x2(a[8 * q + 6] * inv, a[8 * q + 7] * inv));
     }
   }
 }
 
-// kRopeQ: q is un-rotated and the query prologue rotates it (warps 10 and 11).
+// kRopeQ: q is un-rotated; both softmax warpgroups rotate their query tiles in shared memory.
 template <int D, bool kRopeQ>
 __global__ void __launch_bounds__(kThreads, 1)
     window_attn_kernel(const __grid_constant__ CUtensorMap tmq,
@@ -714,25 +694,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(kFull, wait_bounded(&s_full[i], cnt & 1u, g, E));
         if (!ok) break;
         tc_fence_after();
-#if UNSTEP_SOFTMAX_TWO_PASS
-        // pass 1: the row max, reading the scores 32 columns at a time (two buffers: the next
-        // chunk's load is in flight while the current one is reduced)
-        const bool masked = valid < 128;
-        uint32_t bufA[32], bufB[32];
-        tmem_ld32(tS, bufA);
-        tmem_wait_ld_regs(bufA);
-        tmem_ld32(tS + 32, bufB);
-        float mx = chunk_max(bufA, 0, valid, masked);
-        tmem_wait_ld_regs(bufB);
-        tmem_ld32(tS + 64, bufA);
-        mx = fmaxf(mx, chunk_max(bufB, 32, valid, masked));
-        tmem_wait_ld_regs(bufA);
-        tmem_ld32(tS + 96, bufB);
-        mx = fmaxf(mx, chunk_max(bufA, 64, valid, masked));
-        tmem_wait_ld_regs(bufB);
-        mx = fmaxf(mx, chunk_max(bufB, 96, valid, masked));
-        const float mt = mx * scale;
-#else
         uint32_t s[4][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
@@ -746,7 +707,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c * 32 + e >= valid) s[c][e] = __float_as_uint(-INFINITY);
         }
         const float mt = row_max128(s) * scale;
-#endif
         if (j == 0) {
           m_run = mt;
         } else if (__any_sync(kFull, mt > m_run + 8.f)) {
@@ -771,34 +731,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t sc2 = f2_make(scale, scale);
         const uint64_t nm2 = f2_make(-m_run, -m_run);
         uint64_t acc[4] = {0, 0, 0, 0};
-#if UNSTEP_SOFTMAX_TWO_PASS
-        // pass 2: P chunk by chunk; P chunk c goes to columns [16c, 16c + 16), which hold
-        // scores of chunks <= c that are already in registers
-        tmem_ld32(tS, bufA);
-        tmem_wait_ld_regs(bufA);
-        tmem_ld32(tS + 32, bufB);
-        if (!masked) {
-          exp_chunk<false>(bufA, 0, 128, sc2, nm2, acc, tS);
-          tmem_wait_ld_regs(bufB);
-          tmem_ld32(tS + 64, bufA);
-          exp_chunk<false>(bufB, 32, 128, sc2, nm2, acc, tS + 16);
-          tmem_wait_ld_regs(bufA);
-          tmem_ld32(tS + 96, bufB);
-          exp_chunk<false>(bufA, 64, 128, sc2, nm2, acc, tS + 32);
-          tmem_wait_ld_regs(bufB);
-          exp_chunk<false>(bufB, 96, 128, sc2, nm2, acc, tS + 48);
-        } else {
-          exp_chunk<true>(bufA, 0, valid, sc2, nm2, acc, tS);
-          tmem_wait_ld_regs(bufB);
-          tmem_ld32(tS + 64, bufA);
-          exp_chunk<true>(bufB, 32, valid, sc2, nm2, acc, tS + 16);
-          tmem_wait_ld_regs(bufA);
-          tmem_ld32(tS + 96, bufB);
-          exp_chunk<true>(bufA, 64, valid, sc2, nm2, acc, tS + 32);
-          tmem_wait_ld_regs(bufB);
-          exp_chunk<true>(bufB, 96, valid, sc2, nm2, acc, tS + 48);
-        }
-#else
         if (!masked) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -808,7 +740,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 4; ++c)
             exp_chunk<true>(s[c], c * 32, valid, sc2, nm2, acc, tS + c * 16);
         }
-#endif
         float a0, a1;
         f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
         l_run += a0 + a1;
