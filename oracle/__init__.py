@@ -352,3 +352,41 @@ def svd_truncate(W: np.ndarray, rank: int):
 def renoise(x0_bits: np.ndarray, eps_bits: np.ndarray, sigma: float) -> np.ndarray:
     """(1 - sigma) x0 + sigma eps in fp64 from bf16 bit patterns."""
     return (1.0 - sigma) * bf16_to_f64(x0_bits) + sigma * bf16_to_f64(eps_bits)
+
+
+# --------------------------------------------------------------------------------------------
+# Causal 3D convolution of the VAE decoder (abstract: "VAE decoding with optimized memory layout,
+# precision, and convolution kernels"; Table 1 row C2)
+# --------------------------------------------------------------------------------------------
+
+def conv3d_causal(x_bits: np.ndarray, w_bits: np.ndarray,
+                  bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """Causal 3x3x3 convolution in fp64 from bf16 bit patterns, channels-last.
+
+    x: [B][T + 2][H][W][C_in] -- each stream's first two frames are its causal history (the
+    frames the previous chunk ended with, zeros at a stream's start); w: [C_out][3][3][3][C_in]
+    indexed by the taps (dt, dy, dx); bias: [C_out] (fp64) or None.  Output [B][T][H][W][C_out]:
+
+        y[b, t, h, x, o] = bias[o] + sum over dt, dy, dx, c of
+                           w[o, dt, dy, dx, c] * in[b, t + dt, h + dy - 1, x + dx - 1, c]
+
+    with positions outside the frame reading 0 (one position of zero padding in h and w), so that
+    output frame t sees input frames t .. t + 2 (its own frame and the two before it).  Written
+    as the sum over the 27 taps of a shifted slice times the tap's [C_in][C_out] matrix.
+    """
+    x = bf16_to_f64(x_bits)
+    wt = bf16_to_f64(w_bits)
+    B, Tin, H, W, Ci = x.shape
+    Co = wt.shape[0]
+    assert wt.shape == (Co, 3, 3, 3, Ci) and Tin >= 3
+    T = Tin - 2
+    xp = np.zeros((B, Tin, H + 2, W + 2, Ci))
+    xp[:, :, 1:H + 1, 1:W + 1, :] = x
+    y = np.zeros((B, T, H, W, Co))
+    for dt in range(3):
+        for dy in range(3):
+            for dx in range(3):
+                y += xp[:, dt:dt + T, dy:dy + H, dx:dx + W, :] @ wt[:, dt, dy, dx, :].T
+    if bias is not None:
+        y += np.asarray(bias, dtype=np.float64)
+    return y
