@@ -90,6 +90,9 @@ _SIGNATURES = {
                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "unstep_renoise": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong,
                         ctypes.c_float, ctypes.c_void_p], ctypes.c_int),
+    "unstep_conv3d_causal": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                              ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),
@@ -425,6 +428,35 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = No
     _check(lib().unstep_gemm_bf16(_dev_ptr(a, "a"), K, _dev_ptr(b, "b"), K, _dev_ptr(out, "out"),
                                   N, M, N, K, _dev_ptr(err, "dev_error"), _stream_handle(stream)),
            "unstep_gemm_bf16")
+    return out
+
+
+def conv3d_causal(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, dev_error: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal 3x3x3 convolution, channels-last, on the tensor cores.
+
+    x [B][T+2][H][W][C_in] bf16 (each stream's first two frames are its causal history),
+    w [C_out][3][3][3][C_in] bf16, bias [C_out] fp32 or None -> y [B][T][H][W][C_out] bf16.
+    """
+    if x.dtype != torch.bfloat16 or x.dim() != 5 or w.dtype != torch.bfloat16 or w.dim() != 5:
+        raise ValueError("x and w must be 5-D bfloat16 tensors")
+    B, Tin, H, Wd, C_in = x.shape
+    C_out = w.shape[0]
+    if tuple(w.shape[1:]) != (3, 3, 3, C_in):
+        raise ValueError(f"w has shape {tuple(w.shape)}, expected {(C_out, 3, 3, 3, C_in)}")
+    if Tin < 3:
+        raise ValueError("x needs the two history frames and at least one frame")
+    if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (C_out,)):
+        raise ValueError("bias must be float32 [C_out]")
+    if out is None:
+        out = torch.empty((B, Tin - 2, H, Wd, C_out), dtype=torch.bfloat16, device=x.device)
+    err = _err_word(dev_error, x)
+    bp = None if bias is None else _dev_ptr(bias, "bias")
+    _check(lib().unstep_conv3d_causal(_dev_ptr(x, "x"), _dev_ptr(w, "w"), bp, _dev_ptr(out, "out"),
+                                      B, Tin - 2, H, Wd, C_in, C_out, _dev_ptr(err, "dev_error"),
+                                      _stream_handle(stream)),
+           "unstep_conv3d_causal")
     return out
 
 

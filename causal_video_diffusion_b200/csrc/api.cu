@@ -579,6 +579,63 @@ int unstep_renoise(const void *x0, const void *eps, void *out, long long n, floa
   return UNSTEP_OK;
 }
 
+int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *y, int B, int T,
+                         int H, int W, int C_in, int C_out, int *dev_error,
+                         unstep_stream_t stream) {
+  if (!x || !w || !y || !dev_error) return UNSTEP_ERR_ARG;
+  if (B < 1 || T < 1 || H < 1 || W < 1 || C_in < 1 || C_out < 1) return UNSTEP_ERR_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return UNSTEP_ERR_ALIGN;
+  if (C_in % 64 != 0 || C_out % 8 != 0) return UNSTEP_ERR_UNSUPPORTED;
+  const long long frames = static_cast<long long>(B) * (T + 2);
+  const long long tiles_h = (H + 7) / 8, tiles_w = (W + 15) / 16;
+  const long long m_tiles = static_cast<long long>(B) * T * tiles_h * tiles_w;
+  const long long n_tiles = (C_out + 127) / 128;
+  if (frames > 0x7FFFFFFFll || m_tiles * n_tiles > 0x7FFFFFFFll || W > (1 << 24) ||
+      H > (1 << 24) || C_in > (1 << 16) || C_out > (1 << 24))
+    return UNSTEP_ERR_UNSUPPORTED;
+  CUtensorMap tmx, tmw;
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C_in), static_cast<cuuint64_t>(W),
+                                static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(frames)};
+    const cuuint64_t str[3] = {static_cast<cuuint64_t>(C_in) * 2,
+                               static_cast<cuuint64_t>(W) * C_in * 2,
+                               static_cast<cuuint64_t>(H) * W * C_in * 2};
+    const cuuint32_t box[4] = {64, 16, 8, 1};
+    if (!encode_bf16(&tmx, x, 4, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C_in), 27,
+                                static_cast<cuuint64_t>(C_out)};
+    const cuuint64_t str[2] = {static_cast<cuuint64_t>(C_in) * 2,
+                               static_cast<cuuint64_t>(C_in) * 27 * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    if (!encode_bf16(&tmw, w, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
+  unstep::ConvParams p{};
+  p.y = y;
+  p.bias = bias;
+  p.dev_error = dev_error;
+  p.wait_limit_ns = unstep::kWaitLimitNs;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.W = W;
+  p.C_in = C_in;
+  p.C_out = C_out;
+  p.tiles_h = static_cast<int>(tiles_h);
+  p.tiles_w = static_cast<int>(tiles_w);
+  p.m_tiles = static_cast<int>(m_tiles);
+  p.n_tiles = static_cast<int>(n_tiles);
+  if (unstep::launch_conv3d_causal(tmx, tmw, p, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
 int unstep_get_device_error(const unstep_cache_t *cache, unstep_stream_t stream) {
   if (!cache || !cache->dev_error) return UNSTEP_ERR_ARG;
   int v = 0;

@@ -1,0 +1,248 @@
+// conv3d.cu -- the VAE decoder's causal 3D convolution on the Blackwell tensor cores.
+//
+// UnStep paper (arXiv 2609.32518), abstract and Table 1 row C2: the decoder runs with an
+// optimised memory layout, precision and convolution kernels.  The layer here is the causal
+// 3x3x3 convolution of a video decoder, channels-last, bf16 in and out, fp32 accumulation:
+//
+//   y[b, t, h, x, o] = bias[o] + sum over (dt, dy, dx, c) of
+//                      w[o, dt, dy, dx, c] * in[b, t + dt, h + dy - 1, x + dx - 1, c]
+//
+// where each stream's input carries two history frames in front (output frame t sees input
+// frames t .. t + 2) and positions outside the frame read zero.  It is computed as an implicit
+// GEMM: M = output positions, N = output channels, K = 27 taps x C_in.  An output tile is 8 rows
+// x 16 columns of one frame (128 positions) by 128 channels; K advances 64 input channels of one
+// tap at a time, and the A tile of that step is one TMA box {64 channels, 16 x, 8 y, 1 frame} of
+// the input at the tap's offset -- it lands in shared memory as 128 rows of 128 bytes with the
+// 128-byte swizzle, exactly the K-major operand layout, and the box's out-of-range part (the
+// frame's border, the padding) is zero-filled by the TMA unit.  B is the tap's {64 channels x 128
+// output channels} slice of the weights.  The pipeline is the projection GEMM's: a persistent
+// grid, a 6-stage TMA ring, tcgen05.mma M=128 N=128 K=16 into one of two TMEM accumulators, a
+// 4-warp epilogue (thread = TMEM lane = output position) adding the bias and storing bf16.
+#include <cuda_bf16.h>
+
+#include "../../include/unstep.h"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace unstep {
+namespace {
+
+constexpr int kBM = 128, kBN = 128, kBK = 64;
+constexpr int kTileH = 8, kTileW = 16;               // an output tile: 8 rows x 16 columns
+constexpr int kStages = 6;
+constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
+constexpr int kABytes = kBM * kBK * 2;               // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;               // 16 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kSmemBar = kStages * kStageBytes;
+constexpr int kSmemAlloc = kSmemBar + 256 + 1024;
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+// Output tile t -> (n block, frame index b*T + t, first row, first column).
+struct ConvTile {
+  int n0, bt, h0, w0;
+};
+
+__device__ __forceinline__ ConvTile conv_tile(const ConvParams &p, int t) {
+  ConvTile c;
+  const int m = t % p.m_tiles;
+  c.n0 = (t / p.m_tiles) * kBN;
+  c.bt = m / (p.tiles_h * p.tiles_w);
+  const int r = m - c.bt * (p.tiles_h * p.tiles_w);
+  c.h0 = (r / p.tiles_w) * kTileH;
+  c.w0 = (r % p.tiles_w) * kTileW;
+  return c;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    conv3d_causal_kernel(const __grid_constant__ CUtensorMap tmx,
+                         const __grid_constant__ CUtensorMap tmw, const ConvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;   // [2]
+  uint64_t *acc_empty = acc_full + 2;     // [2]
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int ncb = p.C_in / kBK;            // 64-channel blocks per tap
+  const int k_steps = 27 * ncb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard g{abort_flag, p.dev_error, p.wait_limit_ns};
+  constexpr int E = UNSTEP_ERR_DEVICE_TIMEOUT;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmx);
+      tma_prefetch_desc(&tmw);
+      int n = 0;  // stage fills issued
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const ConvTile c = conv_tile(p, t);
+        const int b = c.bt / p.T;
+        const int f0 = c.bt + 2 * b;       // input frame of tap dt = 0 (streams hold T + 2)
+        for (int k = 0; k < k_steps; ++k, ++n) {
+          const int s = n % kStages;
+          const uint32_t r = static_cast<uint32_t>(n / kStages);
+          if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
+          const int tap = k / ncb, c0 = (k - tap * ncb) * kBK;
+          const int dt = tap / 9, dy = (tap / 3) % 3, dx = tap % 3;
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          uint8_t *st = smem + s * kStageBytes;
+          // input box at the tap's offset: x and y may start at -1 (zero fill outside)
+          tma_load_4d(st, &tmx, &full[s], c0, c.w0 + dx - 1, c.h0 + dy - 1, f0 + dt);
+          tma_load_3d(st + kABytes, &tmw, &full[s], c0, tap, c.n0);
+        }
+      }
+      if (*abort_flag)
+        for (int k = max(0, n - kStages); k < n; ++k)
+          drain_wait(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16_f32(kBM, kBN, false, false);
+      const uint32_t hi = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
+      const uint32_t lo0 = static_cast<uint32_t>(sdesc_sw128(smem_u32(smem), 16, 1024));
+      bool ok = true;
+      int n = 0, i = 0;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
+        const int acc = i & 1;
+        if (!(ok = wait_bounded(&acc_empty[acc], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u, g, E)))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * kBN;
+        for (int k = 0; k < k_steps; ++k, ++n) {
+          const int s = n % kStages;
+          if (!(ok = wait_bounded(&full[s], static_cast<uint32_t>(n / kStages) & 1u, g, E))) break;
+          tc_fence_after();
+          const uint32_t la = lo0 + static_cast<uint32_t>((s * kStageBytes) >> 4);
+          const uint32_t lb = la + static_cast<uint32_t>(kABytes >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_ss(d, f2u64(la + kk * 2, hi), f2u64(lb + kk * 2, hi), kId,
+                    (k > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&acc_full[acc]);
+      }
+      umma_commit(drain);
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int row = threadIdx.x - 128;  // TMEM lane = output position of the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const int hh = row / kTileW, ww = row % kTileW;
+    bool ok = true;
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int acc = i & 1;
+      if (ok)
+        ok = __all_sync(kFull, wait_bounded(&acc_full[acc], static_cast<uint32_t>(i >> 1) & 1u, g, E));
+      if (!ok) break;
+      tc_fence_after();
+      const ConvTile c = conv_tile(p, t);
+      const int h = c.h0 + hh, x = c.w0 + ww;
+      const bool live = h < p.H && x < p.W;
+      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) +
+                           ((static_cast<long long>(c.bt) * p.H + h) * p.W + x) * p.C_out;
+      const uint32_t src = tmem + lane_base + acc * kBN;
+#pragma unroll 1
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(src + cc * 32, o);
+        tmem_wait_ld();
+        const int nb = c.n0 + cc * 32;
+        if (live && nb < p.C_out) {
+          float bv[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            bv[e] = (p.bias != nullptr && nb + e < p.C_out) ? __ldg(p.bias + nb + e) : 0.f;
+          uint32_t wv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) + bv[2 * e],
+                                __uint_as_float(o[2 * e + 1]) + bv[2 * e + 1]);
+          const int nv = (p.C_out - nb) >= 32 ? 4 : (p.C_out - nb) / 8;  // 16-byte groups
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (v < nv)
+              reinterpret_cast<uint4 *>(dst + nb)[v] =
+                  make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_conv3d_causal(const CUtensorMap &tmx, const CUtensorMap &tmw,
+                                 const ConvParams &p, cudaStream_t stream) {
+  static unsigned long long attr_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (dev >= 64 || !(__atomic_load_n(&attr_set, __ATOMIC_ACQUIRE) & bit)) {
+    e = cudaFuncSetAttribute(conv3d_causal_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
+  }
+  const long long tiles = static_cast<long long>(p.m_tiles) * p.n_tiles;
+  if (tiles < 1 || tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  conv3d_causal_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(tmx, tmw, p);
+  return cudaGetLastError();
+}
+
+}  // namespace unstep

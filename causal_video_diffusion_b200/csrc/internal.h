@@ -129,6 +129,22 @@ cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cuda
 cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
                                 int N, int K, int ldc, int *dev_error, cudaStream_t stream);
 
+// Causal 3x3x3 convolution (channels-last implicit GEMM); see unstep_conv3d_causal.
+struct ConvParams {
+  void *y;            // bf16 [B][T][H][W][C_out]
+  const float *bias;  // [C_out] or null
+  int *dev_error;
+  uint64_t wait_limit_ns;
+  int B, T, H, W, C_in, C_out;
+  int tiles_h, tiles_w;   // output tiles of 8 rows x 16 columns per frame
+  int m_tiles, n_tiles;   // B*T*tiles_h*tiles_w position tiles; ceil(C_out / 128) channel tiles
+};
+
+// tmx: 4D (C_in, W, H, B*(T+2)) bf16, box (64, 16, 8, 1); tmw: 3D (C_in, 27, C_out) bf16, box
+// (64, 1, 128); both 128B swizzle.
+cudaError_t launch_conv3d_causal(const CUtensorMap &tmx, const CUtensorMap &tmw,
+                                 const ConvParams &p, cudaStream_t stream);
+
 // out[i] = (1 - sigma) * x0[i] + sigma * eps[i], bf16, n elements.
 cudaError_t launch_renoise(const void *x0, const void *eps, void *out, long long n, float sigma,
                            cudaStream_t stream);

@@ -286,6 +286,26 @@ int unstep_renoise(const void *x0, const void *eps, void *out, long long n, floa
                    unstep_stream_t stream);
 
 /*
+ * Causal 3x3x3 convolution of a video VAE decoder, channels-last (the abstract's "VAE decoding
+ * with optimized memory layout, precision, and convolution kernels"; Table 1 row C2).
+ *   x    : bf16 [B][T + 2][H][W][C_in]; each stream's first two frames are its causal history
+ *          (the last two input frames of the previous chunk, or zeros at the stream's start).
+ *   w    : bf16 [C_out][3][3][3][C_in], taps (dt, dy, dx).
+ *   bias : fp32 [C_out], or NULL for none.
+ *   y    : bf16 [B][T][H][W][C_out]; must not overlap x.
+ *   y[b][t][h][x][o] = bias[o] + sum over dt, dy, dx, c of
+ *                      w[o][dt][dy][dx][c] * x[b][t + dt][h + dy - 1][x + dx - 1][c],
+ * positions outside the frame reading 0: output frame t sees input frames t .. t + 2.  bf16
+ * tensor-core products with fp32 accumulation, output rounded to bf16 (RNE).
+ * Errors: ARG (NULL pointer, size < 1), ALIGN (x, w, y not 16-byte aligned, bias not 4-byte),
+ * UNSUPPORTED (C_in not a multiple of 64, C_out not a multiple of 8, sizes beyond the kernel's
+ * 32-bit tile indexing), CUDA.  A device-side wait past its limit sets *dev_error.
+ */
+int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *y, int B, int T,
+                         int H, int W, int C_in, int C_out, int *dev_error,
+                         unstep_stream_t stream);
+
+/*
  * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported
  * an error); CUDA if the copy or the synchronisation itself failed.
  */

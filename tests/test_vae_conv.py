@@ -88,3 +88,22 @@ def test_constant_input_closed_form():
     np.testing.assert_allclose(y[0, :, -1, -1],
                                np.broadcast_to(wf[:, :, :2, :2].sum(axis=(1, 2, 3, 4)),
                                                y[0, :, -1, -1].shape), rtol=1e-12)
+
+
+def test_conv_arguments_rejected_on_the_host():
+    """Every failing call returns before any launch (no GPU needed)."""
+    import ctypes
+    from causal_video_diffusion_b200 import binding as B
+    L = B.lib()
+    p = ctypes.c_void_p(0x700000)
+    odd = ctypes.c_void_p(0x700008)
+    err = ctypes.c_void_p(0x710000)
+    ok_args = (1, 3, 8, 16, 64, 128)
+    f = L.unstep_conv3d_causal
+    assert f(None, p, None, p, *ok_args, err, None) == B.UNSTEP_ERR_ARG
+    assert f(p, p, None, p, *ok_args, None, None) == B.UNSTEP_ERR_ARG
+    assert f(p, p, None, p, 1, 0, 8, 16, 64, 128, err, None) == B.UNSTEP_ERR_ARG
+    assert f(odd, p, None, p, *ok_args, err, None) == B.UNSTEP_ERR_ALIGN
+    assert f(p, p, ctypes.c_void_p(0x700002), p, *ok_args, err, None) == B.UNSTEP_ERR_ALIGN
+    assert f(p, p, None, p, 1, 3, 8, 16, 48, 128, err, None) == B.UNSTEP_ERR_UNSUPPORTED
+    assert f(p, p, None, p, 1, 3, 8, 16, 64, 100, err, None) == B.UNSTEP_ERR_UNSUPPORTED
