@@ -589,7 +589,8 @@ int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *
     return UNSTEP_ERR_ALIGN;
   if (C_in % 64 != 0 || C_out % 8 != 0) return UNSTEP_ERR_UNSUPPORTED;
   const long long frames = static_cast<long long>(B) * (T + 2);
-  const long long tiles_h = (H + 7) / 8, tiles_w = (W + 15) / 16;
+  const long long tiles_h = (H + unstep::kConvTileH - 1) / unstep::kConvTileH;
+  const long long tiles_w = (W + 15) / 16;
   const long long m_tiles = static_cast<long long>(B) * T * tiles_h * tiles_w;
   const long long n_tiles = (C_out + 127) / 128;
   if (frames > 0x7FFFFFFFll || m_tiles * n_tiles > 0x7FFFFFFFll || W > (1 << 24) ||

@@ -9,15 +9,16 @@
 //
 // where each stream's input carries two history frames in front (output frame t sees input
 // frames t .. t + 2) and positions outside the frame read zero.  It is computed as an implicit
-// GEMM: M = output positions, N = output channels, K = 27 taps x C_in.  An output tile is 8 rows
-// x 16 columns of one frame (128 positions) by 128 channels; K advances 64 input channels of one
-// tap at a time, and the A tile of that step is one TMA box {64 channels, 16 x, 8 y, 1 frame} of
-// the input at the tap's offset -- it lands in shared memory as 128 rows of 128 bytes with the
-// 128-byte swizzle, exactly the K-major operand layout, and the box's out-of-range part (the
-// frame's border, the padding) is zero-filled by the TMA unit.  B is the tap's {64 channels x 128
-// output channels} slice of the weights.  The pipeline is the projection GEMM's: a persistent
-// grid, a 6-stage TMA ring, tcgen05.mma M=128 N=128 K=16 into one of two TMEM accumulators, a
-// 4-warp epilogue (thread = TMEM lane = output position) adding the bias and storing bf16.
+// GEMM: M = output positions, N = output channels, K = 27 taps x C_in.  An output tile is 16
+// rows x 16 columns of one frame (two halves of 128 positions) by 128 channels; K advances 64
+// input channels of one tap at a time, and each half's A tile of that step is one TMA box {64
+// channels, 16 x, 8 y, 1 frame} of the input at the tap's offset -- it lands in shared memory as
+// 128 rows of 128 bytes with the 128-byte swizzle, exactly the K-major operand layout, and the
+// box's out-of-range part (the frame's border, the padding) is zero-filled by the TMA unit.  B is
+// the tap's {64 channels x 128 output channels} slice of the weights, shared by both halves.  The
+// pipeline is the projection GEMM's: a persistent grid, a TMA ring, tcgen05.mma M=128 N=128 K=16
+// per half into one of two TMEM accumulator sets, a 4-warp epilogue (thread = TMEM lane = output
+// position of a half) adding the bias and storing bf16.
 #include <cuda_bf16.h>
 
 #include "../../include/unstep.h"
@@ -27,12 +28,19 @@
 namespace unstep {
 namespace {
 
+// kMT 128-position halves per output tile (rows 8 kMT x 16 columns), each its own M=128
+// product against the same weight slice, so that one B load serves kMT x 128 positions
+#ifndef UNSTEP_CONV_MT
+#define UNSTEP_CONV_MT 2
+#endif
+constexpr int kMT = UNSTEP_CONV_MT;
 constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kTileH = 8, kTileW = 16;               // an output tile: 8 rows x 16 columns
-constexpr int kStages = 6;
+constexpr int kTileH = 8 * kMT, kTileW = 16;         // an output tile: 8 kMT rows x 16 columns
+constexpr int kStages = kMT == 1 ? 6 : 4;
 constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
-constexpr int kABytes = kBM * kBK * 2;               // 16 KB
+constexpr int kABytes = kMT * kBM * kBK * 2;         // 16 KB per 128 positions
 constexpr int kBBytes = kBN * kBK * 2;               // 16 KB
+constexpr int kAccCols = kMT * kBN;                  // TMEM columns of one accumulator set
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kSmemBar = kStages * kStageBytes;
 constexpr int kSmemAlloc = kSmemBar + 256 + 1024;
@@ -96,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 2 * kAccCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -125,7 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&full[s], kStageBytes);
           uint8_t *st = smem + s * kStageBytes;
           // input box at the tap's offset: x and y may start at -1 (zero fill outside)
-          tma_load_4d(st, &tmx, &full[s], c0, c.w0 + dx - 1, c.h0 + dy - 1, f0 + dt);
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt)
+            tma_load_4d(st + mt * (kBM * kBK * 2), &tmx, &full[s], c0, c.w0 + dx - 1,
+                        c.h0 + 8 * mt + dy - 1, f0 + dt);
           tma_load_3d(st + kABytes, &tmw, &full[s], c0, tap, c.n0);
         }
       }
@@ -146,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_bounded(&acc_empty[acc], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u, g, E)))
           break;
         tc_fence_after();
-        const uint32_t d = tmem + acc * kBN;
+        const uint32_t d = tmem + acc * kAccCols;
         for (int k = 0; k < k_steps; ++k, ++n) {
           const int s = n % kStages;
           if (!(ok = wait_bounded(&full[s], static_cast<uint32_t>(n / kStages) & 1u, g, E))) break;
@@ -155,8 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t lb = la + static_cast<uint32_t>(kABytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss(d, f2u64(la + kk * 2, hi), f2u64(lb + kk * 2, hi), kId,
-                    (k > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt)
+              umma_ss(d + mt * kBN, f2u64(la + mt * ((kBM * kBK * 2) >> 4) + kk * 2, hi),
+                      f2u64(lb + kk * 2, hi), kId, (k > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&empty[s]);
         }
         if (ok) umma_commit(&acc_full[acc]);
@@ -166,9 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int row = threadIdx.x - 128;  // TMEM lane = output position of the tile
+    const int row = threadIdx.x - 128;  // TMEM lane = output position of a 128-position half
     const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
-    const int hh = row / kTileW, ww = row % kTileW;
+    const int hh = row / 16, ww = row % 16;
     bool ok = true;
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
@@ -178,11 +191,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const ConvTile c = conv_tile(p, t);
-      const int h = c.h0 + hh, x = c.w0 + ww;
+#pragma unroll 1
+      for (int mt = 0; mt < kMT; ++mt) {
+      const int h = c.h0 + 8 * mt + hh, x = c.w0 + ww;
       const bool live = h < p.H && x < p.W;
       __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) +
                            ((static_cast<long long>(c.bt) * p.H + h) * p.W + x) * p.C_out;
-      const uint32_t src = tmem + lane_base + acc * kBN;
+      const uint32_t src = tmem + lane_base + acc * kAccCols + mt * kBN;
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t o[32];
@@ -207,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
         }
       }
+      }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -216,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 2 * kAccCols);
   }
 }
 

@@ -136,9 +136,15 @@ struct ConvParams {
   int *dev_error;
   uint64_t wait_limit_ns;
   int B, T, H, W, C_in, C_out;
-  int tiles_h, tiles_w;   // output tiles of 8 rows x 16 columns per frame
+  int tiles_h, tiles_w;   // output tiles of kConvTileH rows x 16 columns per frame
   int m_tiles, n_tiles;   // B*T*tiles_h*tiles_w position tiles; ceil(C_out / 128) channel tiles
 };
+
+// Rows of a convolution output tile (two 8 x 16 halves of 128 positions).
+#ifndef UNSTEP_CONV_MT
+#define UNSTEP_CONV_MT 2
+#endif
+constexpr int kConvTileH = 8 * UNSTEP_CONV_MT;
 
 // tmx: 4D (C_in, W, H, B*(T+2)) bf16, box (64, 16, 8, 1); tmw: 3D (C_in, 27, C_out) bf16, box
 // (64, 1, 128); both 128B swizzle.
