@@ -19,10 +19,16 @@
 namespace unstep {
 namespace {
 
+// kMT 128-row halves per output tile, each its own M=128 product against the same B tile
+#ifndef UNSTEP_GEMM_MT
+#define UNSTEP_GEMM_MT 2
+#endif
+constexpr int kMT = UNSTEP_GEMM_MT;
 constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kStages = 6;
+constexpr int kStages = kMT == 1 ? 6 : 4;
 constexpr int kThreads = 256;                       // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
-constexpr int kABytes = kBM * kBK * 2;              // 16 KB
+constexpr int kABytes = kMT * kBM * kBK * 2;        // 16 KB per 128 rows
+constexpr int kAccCols = kMT * kBN;                 // TMEM columns of one accumulator set
 constexpr int kBBytes = kBN * kBK * 2;              // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kSmemBar = kStages * kStageBytes;
@@ -66,7 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m_tiles = (M + kBM - 1) / kBM;
+  const int m_tiles = (M + kMT * kBM - 1) / (kMT * kBM);
   const int n_tiles = (N + kBN - 1) / kBN;
   const int tiles = m_tiles * n_tiles;
   const int k_steps = (K + kBK - 1) / kBK;
@@ -85,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 2 * kAccCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -102,14 +108,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = 0;  // stage fills issued
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const int m0 = (t % m_tiles) * kBM, n0 = (t / m_tiles) * kBN;
+        const int m0 = (t % m_tiles) * (kMT * kBM), n0 = (t / m_tiles) * kBN;
         for (int k = 0; k < k_steps; ++k, ++n) {
           const int s = n % kStages;
           const uint32_t r = static_cast<uint32_t>(n / kStages);
           if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
           mbar_arrive_expect_tx(&full[s], kStageBytes);
           uint8_t *st = smem + s * kStageBytes;
-          tma_load_2d(st, &tma, &full[s], k * kBK, m0);
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt)
+            tma_load_2d(st + mt * (kBM * kBK * 2), &tma, &full[s], k * kBK, m0 + mt * kBM);
           tma_load_2d(st + kABytes, &tmb, &full[s], k * kBK, n0);
         }
       }
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_bounded(&acc_empty[acc], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u, g, E)))
           break;
         tc_fence_after();
-        const uint32_t d = tmem + acc * kBN;
+        const uint32_t d = tmem + acc * kAccCols;
         for (int k = 0; k < k_steps; ++k, ++n) {
           const int s = n % kStages;
           if (!(ok = wait_bounded(&full[s], static_cast<uint32_t>(n / kStages) & 1u, g, E))) break;
@@ -139,8 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t lb = la + static_cast<uint32_t>(kABytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss(d, f2u64(la + kk * 2, hi), f2u64(lb + kk * 2, hi), kId,
-                    (k > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt)
+              umma_ss(d + mt * kBN, f2u64(la + mt * ((kBM * kBK * 2) >> 4) + kk * 2, hi),
+                      f2u64(lb + kk * 2, hi), kId, (k > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&empty[s]);
         }
         if (ok) umma_commit(&acc_full[acc]);
@@ -159,8 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(kFull, wait_bounded(&acc_full[acc], static_cast<uint32_t>(i >> 1) & 1u, g, E));
       if (!ok) break;
       tc_fence_after();
-      const int m = (t % m_tiles) * kBM + row, n0 = (t / m_tiles) * kBN;
-      const uint32_t src = tmem + lane_base + acc * kBN;
+#pragma unroll 1
+      for (int mt = 0; mt < kMT; ++mt) {
+      const int m = (t % m_tiles) * (kMT * kBM) + mt * kBM + row, n0 = (t / m_tiles) * kBN;
+      const uint32_t src = tmem + lane_base + acc * kAccCols + mt * kBN;
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t o[32];
@@ -181,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
+      }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -190,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 2 * kAccCols);
   }
 }
 
@@ -209,7 +222,8 @@ cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, vo
     if (e != cudaSuccess) return e;
     if (dev < 64) __atomic_fetch_or(&attr_set, bit, __ATOMIC_RELEASE);
   }
-  const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+  const long long tiles =
+      static_cast<long long>((M + kMT * kBM - 1) / (kMT * kBM)) * ((N + kBN - 1) / kBN);
   if (tiles < 1 || tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

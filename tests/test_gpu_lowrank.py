@@ -36,7 +36,8 @@ def test_gemm_matches_oracle(M, N, K):
 
 
 def test_lowrank_projection_wan_shape():
-    """V projection of the Wan layer through its rank-1413 (padded 1416) factors, 4680 tokens."""
+    """V projection of the Wan layer through its rank-1413 (stored padded to 1472) factors, 4680
+    tokens."""
     d, M = W.MODEL_DIM, 4680
     r = lowrank.retained_rank(d)
     Wt = W.gen_weight(21, d, d)

@@ -14,7 +14,8 @@ from causal_video_diffusion_b200 import workloads as W
 def test_rank_reading_of_the_pages():
     # Figure 11 / Table 5: V/O rank retention fixed at 0.92 of the 1536-wide projections
     assert lowrank.retained_rank(1536) == 1413
-    assert lowrank.padded(1413) == 1416
+    assert lowrank.padded(1413) == 1472    # zero factors up to 128-byte rows
+    assert lowrank.padded(1413, 8) == 1416
 
 
 def test_eckart_young_error_of_the_truncation():
@@ -42,15 +43,18 @@ def test_matmul_against_loops():
 def test_product_factors_match_the_oracle_truncation():
     """The product helper's bf16 factors reproduce the oracle's rank-r weight (up to bf16)."""
     Wt = W.gen_weight(3, 64, 48)
-    w1, w2 = lowrank.svd_factors(Wt, 40)
+    w1, w2 = lowrank.svd_factors(Wt, 40, pad_to=8)
     assert w1.shape == (40, 48) and w2.shape == (64, 40)
     o1, o2, _ = oracle.svd_truncate(Wt.double().numpy(), 40)
     prod = w2.double().numpy() @ w1.double().numpy()
     ref = o2 @ o1
     assert np.max(np.abs(prod - ref)) < 2e-2 * np.max(np.abs(ref))
-    # padding to a multiple of 8 adds zero factors only
-    p1, p2 = lowrank.svd_factors(Wt, 37)
+    # padding (to a multiple of 8 here, of 64 by default) adds zero factors only
+    p1, p2 = lowrank.svd_factors(Wt, 37, pad_to=8)
     assert p1.shape == (40, 48) and torch.all(p1[37:] == 0) and torch.all(p2[:, 37:] == 0)
+    d1, d2 = lowrank.svd_factors(Wt, 37)
+    assert d1.shape == (64, 48) and d2.shape == (64, 64)
+    assert torch.equal(d1[:40], p1) and torch.all(d1[40:] == 0) and torch.equal(d2[:, :40], p2)
 
 
 def test_gemm_arguments_rejected_on_the_host():
