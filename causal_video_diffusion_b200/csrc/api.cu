@@ -550,8 +550,17 @@ int unstep_gemm_bf16(const void *a, int lda, const void *b, int ldb, void *c, in
     const cuuint32_t box[2] = {64, 128};
     if (!encode_bf16(&tb, b, 2, dims, str, box)) return UNSTEP_ERR_CUDA;
   }
-  if (unstep::launch_gemm_bf16_tn(ta, tb, c, M, N, K, ldc, dev_error,
-                                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+  // CTA pairs (256 x 256 tiles) when the product is at least one pair tile; else single CTAs
+#ifndef UNSTEP_GEMM_2SM
+#define UNSTEP_GEMM_2SM 1
+#endif
+  const bool pair = UNSTEP_GEMM_2SM && M >= 256 && N >= 256;
+  const cudaError_t e =
+      pair ? unstep::launch_gemm2sm_bf16_tn(ta, tb, c, M, N, K, ldc, dev_error,
+                                            reinterpret_cast<cudaStream_t>(stream))
+           : unstep::launch_gemm_bf16_tn(ta, tb, c, M, N, K, ldc, dev_error,
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
   }

@@ -129,6 +129,10 @@ cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cuda
 cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
                                 int N, int K, int ldc, int *dev_error, cudaStream_t stream);
 
+// The same product on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles); same tensor maps.
+cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
+                                   int N, int K, int ldc, int *dev_error, cudaStream_t stream);
+
 // Causal 3x3x3 convolution (channels-last implicit GEMM); see unstep_conv3d_causal.
 struct ConvParams {
   void *y;            // bf16 [B][T][H][W][C_out]
