@@ -468,7 +468,8 @@ def run_lowrank(args, rank, local_rank, world):
                                f"(stored padded to {r}), V then O",
                    "l2": "flushed between steps"},
         "gpu_launches": 4 * args.steps,
-        "roofline": {"kernel": "gemm_bf16_tn_kernel", "bound": "tensor", "achieved": round(tf, 2),
+        "roofline": {"kernel": "gemm2sm_bf16_tn_kernel (CTA pairs)", "bound": "tensor",
+                     "achieved": round(tf, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": src}}),
         flush=True)
