@@ -370,10 +370,17 @@ def cpu_baseline(wl, q, k, v, cache, args):
     oracle.set_num_threads(cores)
     qb, kb, vb = (W.bits(t.cpu()) for t in (q, k, v))
     step_s, measured, sample = _oracle_sample(wl, qb, kb, vb, [0, wl.shape.H - 1], args.cpu_rows)
+    used = oracle.num_threads()
     flops = wl.attn_flops(wl.chunks - 1)
+    # the same oracle on one thread, on a smaller sample of the same step
+    oracle.set_num_threads(1)
+    step1_s, measured1, sample1 = _oracle_sample(wl, qb, kb, vb, [0], max(1, args.cpu_rows // 64))
+    oracle.set_num_threads(cores)
     return {"value": round(flops / step_s / 1e12, 6), "unit": "TFLOP/s",
-            "cores": oracle.num_threads(), "kind": "oracle", "sample": sample,
-            "seconds_measured": round(measured, 3), "extrapolated_step_s": round(step_s, 3)}
+            "cores": used, "kind": "oracle", "sample": sample,
+            "seconds_measured": round(measured, 3), "extrapolated_step_s": round(step_s, 3),
+            "value_1thread": round(flops / step1_s / 1e12, 6), "sample_1thread": sample1,
+            "seconds_measured_1thread": round(measured1, 3)}
 
 
 def run_reference(args, rank, world):
@@ -596,7 +603,8 @@ def main():
                     help="wan_full (default), wan_window, long_b4, wan_full_h8, tiny; or the "
                          "separate legs lowrank_vo, clip30, vae_conv")
     ap.add_argument("--seed", type=int, default=2024)
-    ap.add_argument("--cpu-rows", type=int, default=1024, help="oracle rows per head (baseline)")
+    ap.add_argument("--cpu-rows", type=int, default=8192,
+                    help="oracle rows per head of the CPU baseline (about 10 s on 16 cores)")
     ap.add_argument("--ref-rows", type=int, default=32, help="oracle rows per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-rope", choices=["append", "attn"], default="append",
