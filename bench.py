@@ -369,7 +369,9 @@ def cpu_baseline(wl, q, k, v, cache, args):
     cores = len(os.sched_getaffinity(0))
     oracle.set_num_threads(cores)
     qb, kb, vb = (W.bits(t.cpu()) for t in (q, k, v))
-    step_s, measured, sample = _oracle_sample(wl, qb, kb, vb, [0, wl.shape.H - 1], args.cpu_rows)
+    H = wl.shape.H
+    heads = sorted({0, H // 3, (2 * H) // 3, H - 1})   # four heads at the shape benchmarked
+    step_s, measured, sample = _oracle_sample(wl, qb, kb, vb, heads, args.cpu_rows)
     used = oracle.num_threads()
     flops = wl.attn_flops(wl.chunks - 1)
     # the same oracle on one thread, on a smaller sample of the same step
@@ -604,7 +606,7 @@ def main():
                          "separate legs lowrank_vo, clip30, vae_conv")
     ap.add_argument("--seed", type=int, default=2024)
     ap.add_argument("--cpu-rows", type=int, default=8192,
-                    help="oracle rows per head of the CPU baseline (about 10 s on 16 cores)")
+                    help="oracle rows per head (at most the chunk's queries) of the CPU baseline")
     ap.add_argument("--ref-rows", type=int, default=32, help="oracle rows per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-rope", choices=["append", "attn"], default="append",
