@@ -6,7 +6,8 @@
   scores depend only on position differences);
 * the ring cache + window attention against a brute force that keeps all frames and masks, and
   against torch's fp64 ``scaled_dot_product_attention``;
-* closed forms of attention: constant V, q = 0 gives the plain mean of V over exactly the window.
+* closed forms of attention: constant V, q = 0 gives the plain mean of V over exactly the window;
+* the key order: the ring's physical slot order gives the oldest-first result.
 """
 import math
 import os
@@ -318,6 +319,35 @@ def test_zero_query_gives_window_mean():
         assert np.allclose(out[:, 0], 1.0, atol=1e-14)
         assert np.allclose(out[:, 1], np.mean(frames), atol=1e-12)
         assert np.allclose(out[:, 2], np.mean(np.arange(Tf) % 256) / 256, atol=1e-14)
+
+
+@pytest.mark.parametrize("cap,window,chunks", [(6, 6, 5), (9, 6, 4), (9, 9, 7)])
+def test_physical_slot_order_gives_the_logical_result(cap, window, chunks):
+    """Attending the window's keys in the ring's physical slot order (how the cache lies in
+    memory, and the order a kernel walks it) gives the oldest-first result up to rounding:
+    softmax attention is a sum over keys, so the order of the keys cannot matter."""
+    B, H, Hg, Wg, F, D = 1, 2, 3, 4, 3, 64
+    ol = oracle.OracleLayer(B, H, Hg, Wg, oracle.RopeSpec(24, 20, 20, 10000.0), cap)
+    rng = np.random.default_rng(11)
+    for c in range(chunks):
+        q, k, v = (oracle.f64_to_bf16(rng.normal(size=(B, F * Hg * Wg, H, D))) for _ in range(3))
+        q_rot = ol.append(q, k, v, c * F, F)
+    logical = ol.attend(q_rot, window)
+    Tf = Hg * Wg
+    slots_logical = [ol.slot_of(f) for f in ol.window_frames(window)]
+    slots_physical = sorted(slots_logical)
+    assert slots_physical != slots_logical        # the window wraps the ring in these cases
+    idx = np.concatenate([np.arange(s * Tf, (s + 1) * Tf) for s in slots_physical])
+    rows = [(b, l, h) for b in range(B) for h in range(H) for l in range(F * Tf)]
+    physical = oracle.attention_rows(q_rot, ol.K[:, :, idx, :], ol.V[:, :, idx, :], rows,
+                                     1.0 / math.sqrt(D))
+    np.testing.assert_allclose(physical, logical, rtol=1e-12, atol=1e-14)
+    # a permutation that is not a reordering of whole keys (one value row moved to another key)
+    # must not pass the same check
+    bad_v = ol.V[:, :, idx, :].copy()
+    bad_v[:, :, [0, 1]] = bad_v[:, :, [1, 0]]
+    wrong = oracle.attention_rows(q_rot, ol.K[:, :, idx, :], bad_v, rows, 1.0 / math.sqrt(D))
+    assert np.max(np.abs(wrong - logical)) > 1e-6
 
 
 # ------------------------------------------------------------------------------------------
