@@ -88,18 +88,19 @@ def test_streams_match_oracle(D, split, Hg, Wg, frames, cap, window, chunks, sta
     _run_stream(shape, cap, window, sched, seed=D + Hg * 7 + cap, use_scratch=use_scratch)
 
 
+@pytest.mark.parametrize("D,split", [(64, (24, 20, 20)), (128, (44, 42, 42))])
 @pytest.mark.parametrize("extra", [1, 2, 5])
-def test_tail_units_split_into_many_pieces(extra):
+def test_tail_units_split_into_many_pieces(extra, D, split):
     """One full data-parallel wave plus a tail of 1, 2 or 5 units: each tail unit's key tiles are
     cut over up to 8 CTAs, and the last finisher of each query tile merges up to 8 pieces."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     # one 192-query chunk (one unit of two query tiles per head) over 16 frames of 64 tokens:
     # 8 key tiles per unit, sms + extra units
-    shape = W.LayerShape(B=1, H=sms + extra, D=64, Hg=8, Wg=8, d_t=24, d_h=20, d_w=20,
-                         chunk_frames=3)
+    shape = W.LayerShape(B=1, H=sms + extra, D=D, Hg=8, Wg=8, d_t=split[0], d_h=split[1],
+                         d_w=split[2], chunk_frames=3)
     sched = [(3 * c, 3) for c in range(6)]      # frames 0 .. 17; the last chunk sees 16 frames
     heads = sorted(set(range(0, shape.H, 7)) | set(range(sms - 1, shape.H)))  # all tail units
-    _run_stream(shape, 16, 16, sched, seed=40 + extra, check_cache=False, heads=heads)
+    _run_stream(shape, 16, 16, sched, seed=40 + extra + D, check_cache=False, heads=heads)
 
 
 def _structured_v(shape, f0):
