@@ -46,6 +46,8 @@ def _check(got, x_bits, w_bits, bias, want, row=None):
     (2, 2, 8, 16, 128, 200),    # exactly one position tile per frame, C_out = 128 + 72
     (1, 1, 5, 7, 192, 64),      # a frame smaller than one tile, 3 channel blocks, C_out < 128
     (1, 2, 17, 33, 64, 264),    # 3 x 3 tiles with 1-wide tails, 3 channel tiles (one of 8)
+    (1, 9, 60, 104, 64, 256),   # 504 tiles: 3-4 per persistent CTA, both accumulator sets
+                                # through both barrier phases
 ])
 def test_conv_matches_oracle(B, T, H, Wd, Ci, Co):
     x, w, bias = _inputs(B, T, H, Wd, Ci, Co, seed=B * 1000 + H * 10 + Co)

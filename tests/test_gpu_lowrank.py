@@ -18,7 +18,10 @@ def _rel_errors(got, want):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 8, 8), (300, 136, 1416), (4680, 1416, 1536),
-                                   (257, 520, 72), (129, 264, 200)])
+                                   (257, 520, 72), (129, 264, 200),
+                                   # 3-4 tiles per persistent pair / CTA: both accumulator sets
+                                   # of each go through both barrier phases
+                                   (4096, 4096, 128), (65536, 200, 64)])
 def test_gemm_matches_oracle(M, N, K):
     a = W.gen_act(M * 7 + 1, M, K)
     b = W.gen_act(N * 11 + 2, N, K)
