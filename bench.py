@@ -73,27 +73,42 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_digest() -> str:
+ATTN_SOURCES = ("window_attn.cu", "sm100.cuh", "internal.h")
+GEMM_SOURCES = ("gemm2sm.cu", "sm100.cuh", "internal.h")
+CONV_SOURCES = ("conv3d.cu", "sm100.cuh", "internal.h")
+
+
+def source_digest(names=ATTN_SOURCES) -> str:
+    """Digest of a kernel's source files, as the ncu summaries in profiles/ record it."""
     h = hashlib.sha256()
-    for name in ("window_attn.cu", "sm100.cuh", "internal.h"):
+    for name in names:
         with open(os.path.join(ROOT, "causal_video_diffusion_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def kernel_source_digest() -> str:
+    return source_digest(ATTN_SOURCES)
+
+
+def profile_traffic(profile: str, names):
+    """DRAM bytes per launch recorded in profiles/<profile>, if it was taken on the current
+    source of the kernel (else None)."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source:\s*([0-9a-f]+)", text)
+    if not m or m.group(2) != source_digest(names):
+        return None
+    return float(m.group(1))
 
 
 def profiled_traffic(workload: str, rope_q: bool = False):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
     current kernel source (else None); ``rope_q``: the instantiation with the query prologue."""
     name = f"window_attn_qrope_{workload}.txt" if rope_q else f"window_attn_{workload}.txt"
-    path = os.path.join(ROOT, "profiles", name)
-    try:
-        text = open(path).read()
-    except OSError:
-        return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source:\s*([0-9a-f]+)", text)
-    if not m or m.group(2) != kernel_source_digest():
-        return None
-    return float(m.group(1))
+    return profile_traffic(name, ATTN_SOURCES)
 
 
 class ClockSampler:
@@ -457,10 +472,14 @@ def run_lowrank(args, rank, local_rank, world):
     for _ in range(args.warmup):
         step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
     torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for e in evs:
         step(e)
     torch.cuda.synchronize()
+    clocks = sampler.stop()
     if int(err.item()) != 0:
         raise RuntimeError("device error in the projections")
     ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
@@ -476,12 +495,37 @@ def run_lowrank(args, rank, local_rank, world):
         "config": {"workload": f"lowrank_vo: M={M} d={d} rank={lowrank.retained_rank(d)} "
                                f"(stored padded to {r}), V then O",
                    "l2": "flushed between steps"},
+        "scaling": "weak", "vs_baseline": None,
         "gpu_launches": 4 * args.steps,
         "roofline": {"kernel": "gemm2sm_bf16_tn_kernel (CTA pairs)", "bound": "tensor",
                      "achieved": round(tf, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": src}}),
+                     "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": src,
+                     "traffic": profile_traffic("gemm_bf16_lowrank_vo.txt", GEMM_SOURCES)},
+        "clocks": clocks,
+        "cpu_baseline": None if args.no_cpu_baseline else
+        _lowrank_cpu_baseline(x, facs, flops, M)}),
         flush=True)
+
+
+def _lowrank_cpu_baseline(x, facs, flops, M, rows=None):
+    """The fp64 oracle of the same four products on ``rows`` tokens (default all M),
+    extrapolated to M."""
+    import oracle
+    from causal_video_diffusion_b200 import workloads as W
+    rows = M if rows is None else rows
+    xb = W.bits(x[:rows].cpu())
+    (a1, a2), (b1, b2) = [(W.bits(f1.cpu()), W.bits(f2.cpu())) for f1, f2 in facs]
+    t0 = time.perf_counter()
+    yv = oracle.lowrank_linear(xb, a1, a2)
+    oracle.lowrank_linear(oracle.f64_to_bf16(yv), b1, b2)
+    dt = time.perf_counter() - t0
+    step_s = dt * M / rows
+    return {"value": round(flops / step_s / 1e12, 6), "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"the V and O projections of {rows} of {M} tokens in fp64 (numpy)"
+                      + (", extrapolated to the whole step" if rows < M else ""),
+            "seconds_measured": round(dt, 3)}
 
 
 def run_vae_conv(args, rank, local_rank, world):
@@ -514,10 +558,14 @@ def run_vae_conv(args, rank, local_rank, world):
     for _ in range(args.warmup):
         step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
     torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for e in evs:
         step(e)
     torch.cuda.synchronize()
+    clocks = sampler.stop()
     if int(err.item()) != 0:
         raise RuntimeError("device error in the convolution")
     ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
@@ -531,11 +579,35 @@ def run_vae_conv(args, rank, local_rank, world):
         "dtype": "bf16", "data": "synthetic N(0,1) activations, N(0,1/(27 C)) weights",
         "config": {"workload": f"vae_conv: B={B} T={T}(+2 history) H={H} W={Wd} C_in={C} "
                                f"C_out={C}, channels-last", "l2": "flushed between steps"},
+        "scaling": "weak", "vs_baseline": None,
         "gpu_launches": args.steps,
         "roofline": {"kernel": "conv3d_causal_kernel", "bound": "tensor", "achieved": round(tf, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": src,
-                     "flops_per_launch": flops}}), flush=True)
+                     "flops_per_launch": flops,
+                     "traffic": profile_traffic("conv3d_vae_conv.txt", CONV_SOURCES)},
+        "clocks": clocks,
+        "cpu_baseline": None if args.no_cpu_baseline else
+        _conv_cpu_baseline(x, w, bias, flops, H)}), flush=True)
+
+
+def _conv_cpu_baseline(x, w, bias, flops, H, rows=None):
+    """The fp64 oracle of the same layer on a band of ``rows`` output rows (default all H),
+    extrapolated."""
+    import oracle
+    from causal_video_diffusion_b200 import workloads as W
+    rows = H if rows is None else rows
+    xb = W.bits(x[:, :, :rows].cpu())
+    wb = W.bits(w.cpu())
+    t0 = time.perf_counter()
+    oracle.conv3d_causal(xb, wb, bias.double().cpu().numpy())
+    dt = time.perf_counter() - t0
+    step_s = dt * H / rows
+    return {"value": round(flops / step_s / 1e12, 6), "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{rows} of {H} output rows of every frame and channel in fp64 (numpy)"
+                      + (", extrapolated to the whole layer" if rows < H else ""),
+            "seconds_measured": round(dt, 3)}
 
 
 def run_clip(args, rank, local_rank, world):
