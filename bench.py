@@ -663,7 +663,13 @@ def run_clip(args, rank, local_rank, world):
         "eager_ms_per_clip": round(eager_ms, 3),
         "chunk_steps_per_s": round(drv.calls / (graph_ms * 1e-3), 1),
         "attention_only_frames_per_s": round(81 / (graph_ms * 1e-3), 1),
+        "scaling": "weak", "vs_baseline": None,
         "gpu_launches": (2 * drv.layers + 1) * len(drv.sched),
+        "roofline": {"kernel": "window_attn_kernel<128, false> (with the RoPE+append and renoise "
+                               "launches of every forward)", "bound": "tensor",
+                     "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": src,
+                     "traffic": None},
         "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "clocks": clocks}), flush=True)
 
 
