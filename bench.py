@@ -544,6 +544,7 @@ def run_vae_conv(args, rank, local_rank, world):
     bias = torch.randn((C,), generator=g, device=dev, dtype=torch.float32) * 0.1
     y = torch.empty((B, T, H, Wd, C), dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    scratch = binding.conv3d_scratch(dev)   # stream-K tail over the SMs
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -552,7 +553,7 @@ def run_vae_conv(args, rank, local_rank, world):
         flush.zero_()
         flush_r.sum()
         ev[0].record(stream)
-        binding.conv3d_causal(x, w, bias, out=y, dev_error=err)
+        binding.conv3d_causal(x, w, bias, out=y, dev_error=err, scratch=scratch)
         ev[1].record(stream)
 
     for _ in range(args.warmup):

@@ -92,7 +92,9 @@ _SIGNATURES = {
                         ctypes.c_float, ctypes.c_void_p], ctypes.c_int),
     "unstep_conv3d_causal": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                              ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+                              ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                              ctypes.c_void_p], ctypes.c_int),
+    "unstep_conv3d_scratch_bytes": ([], ctypes.c_size_t),
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),
@@ -431,13 +433,27 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = No
     return out
 
 
+def conv3d_scratch(device: Optional[torch.device] = None) -> torch.Tensor:
+    """A zero-filled scratch buffer for conv3d_causal's stream-K tail on `device` (its size
+    depends on the device's SM count only).  Calls sharing one buffer must be ordered."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        need = int(lib().unstep_conv3d_scratch_bytes())
+    if need <= 0:
+        raise UnstepError(UNSTEP_ERR_CUDA, "unstep_conv3d_scratch_bytes")
+    return torch.zeros((need,), dtype=torch.uint8, device=dev)
+
+
 def conv3d_causal(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
                   out: Optional[torch.Tensor] = None, dev_error: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                  stream: Optional[torch.cuda.Stream] = None,
+                  scratch: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Causal 3x3x3 convolution, channels-last, on the tensor cores.
 
     x [B][T+2][H][W][C_in] bf16 (each stream's first two frames are its causal history),
     w [C_out][3][3][3][C_in] bf16, bias [C_out] fp32 or None -> y [B][T][H][W][C_out] bf16.
+    scratch: a conv3d_scratch() buffer to split the last partial wave of tiles over all SMs
+    (stream-K), or None to run every tile whole.
     """
     if x.dtype != torch.bfloat16 or x.dim() != 5 or w.dtype != torch.bfloat16 or w.dim() != 5:
         raise ValueError("x and w must be 5-D bfloat16 tensors")
@@ -453,9 +469,12 @@ def conv3d_causal(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor]
         out = torch.empty((B, Tin - 2, H, Wd, C_out), dtype=torch.bfloat16, device=x.device)
     err = _err_word(dev_error, x)
     bp = None if bias is None else _dev_ptr(bias, "bias")
+    sp, sb = None, 0
+    if scratch is not None:
+        sp, sb = _dev_ptr(scratch, "scratch"), scratch.numel() * scratch.element_size()
     _check(lib().unstep_conv3d_causal(_dev_ptr(x, "x"), _dev_ptr(w, "w"), bp, _dev_ptr(out, "out"),
-                                      B, Tin - 2, H, Wd, C_in, C_out, _dev_ptr(err, "dev_error"),
-                                      _stream_handle(stream)),
+                                      B, Tin - 2, H, Wd, C_in, C_out, sp, sb,
+                                      _dev_ptr(err, "dev_error"), _stream_handle(stream)),
            "unstep_conv3d_causal")
     return out
 

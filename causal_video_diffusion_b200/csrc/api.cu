@@ -588,14 +588,26 @@ int unstep_renoise(const void *x0, const void *eps, void *out, long long n, floa
   return UNSTEP_OK;
 }
 
+size_t unstep_conv3d_scratch_bytes(void) {
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  return unstep::conv_scratch_bytes(sms);
+}
+
 int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *y, int B, int T,
-                         int H, int W, int C_in, int C_out, int *dev_error,
-                         unstep_stream_t stream) {
+                         int H, int W, int C_in, int C_out, void *scratch, size_t scratch_bytes,
+                         int *dev_error, unstep_stream_t stream) {
   if (!x || !w || !y || !dev_error) return UNSTEP_ERR_ARG;
   if (B < 1 || T < 1 || H < 1 || W < 1 || C_in < 1 || C_out < 1) return UNSTEP_ERR_ARG;
-  if (!aligned16(x) || !aligned16(w) || !aligned16(y) ||
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || !aligned16(scratch) ||
       (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
     return UNSTEP_ERR_ALIGN;
+  int sms = 0;
+  if (scratch) {
+    sms = device_sms();
+    if (sms <= 0) return UNSTEP_ERR_CUDA;
+    if (scratch_bytes < unstep::conv_scratch_bytes(sms)) return UNSTEP_ERR_ARG;
+  }
   if (C_in % 64 != 0 || C_out % 8 != 0) return UNSTEP_ERR_UNSUPPORTED;
   const long long frames = static_cast<long long>(B) * (T + 2);
   const long long tiles_h = (H + unstep::kConvTileH - 1) / unstep::kConvTileH;
@@ -638,6 +650,12 @@ int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *
   p.tiles_w = static_cast<int>(tiles_w);
   p.m_tiles = static_cast<int>(m_tiles);
   p.n_tiles = static_cast<int>(n_tiles);
+  if (scratch) {
+    p.counters = static_cast<unsigned *>(scratch);
+    p.slots = reinterpret_cast<float *>(static_cast<char *>(scratch) +
+                                        unstep::conv_counter_bytes(sms));
+    p.epoch = next_epoch();
+  }
   if (unstep::launch_conv3d_causal(tmx, tmw, p, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
     cudaGetLastError();

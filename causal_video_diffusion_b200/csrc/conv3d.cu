@@ -18,7 +18,8 @@
 // the tap's {64 channels x 128 output channels} slice of the weights, shared by both halves.  The
 // pipeline is the projection GEMM's: a persistent grid, a TMA ring, tcgen05.mma M=128 N=128 K=16
 // per half into one of two TMEM accumulator sets, a 4-warp epilogue (thread = TMEM lane = output
-// position of a half) adding the bias and storing bf16.
+// position of a half) adding the bias and storing bf16.  With caller scratch, the tiles of the
+// last, partial wave are cut along K over all SMs (stream-K, below).
 #include <cuda_bf16.h>
 
 #include "../../include/unstep.h"
@@ -71,6 +72,85 @@ __device__ __forceinline__ ConvTile conv_tile(const ConvParams &p, int t) {
   return c;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Work list of CTA c.  The grid is persistent.  Without a stream-K tail (g_sk = 0) CTA c takes
+// tiles c, c + grid, ... whole.  With one, it first takes its share [lo, hi) of the tail tiles'
+// K steps (at most two pieces, as a share is never longer than one tile), then whole tiles
+// w*grid + c below tail0.  The tail comes first so that the merges of split tiles overlap the
+// whole tiles' main loops instead of ending the launch.  A piece that is not a whole tile leaves
+// its fp32 sums in slot 2c + (piece index); the last of a tile's pieces to finish (an atomic
+// count per tile) adds the others' slots to its own accumulator and stores the tile.  No CTA
+// waits for another.
+// ---------------------------------------------------------------------------------------------
+struct ConvItem {
+  int t;        // output tile
+  int k0, k1;   // K steps [k0, k1) of the tile
+  int slot;     // scratch slot of a partial piece, -1 when the tile is whole
+  long long s0; // first K step of the tile in the tail's numbering (partial pieces only)
+};
+
+__device__ __forceinline__ long long conv_sk_lo(const ConvParams &p, int c) {
+  return static_cast<long long>(c) * p.w_tail / p.g_sk;
+}
+
+struct ConvList {
+  long long lo, hi;
+  int n_sk;    // tail pieces of this CTA
+  int dp_end;  // whole tiles are those below dp_end
+};
+
+__device__ __forceinline__ ConvList conv_list(const ConvParams &p, int c, int k_steps) {
+  ConvList l{0, 0, 0, p.m_tiles * p.n_tiles};
+  if (p.g_sk > 0) {
+    l.dp_end = p.tail0;
+    if (c < p.g_sk) {
+      l.lo = conv_sk_lo(p, c);
+      l.hi = conv_sk_lo(p, c + 1);
+      if (l.hi > l.lo) l.n_sk = static_cast<int>((l.hi - 1) / k_steps - l.lo / k_steps) + 1;
+    }
+  }
+  return l;
+}
+
+// The q-th item of CTA c; false past the last one.
+__device__ __forceinline__ bool conv_item(const ConvParams &p, const ConvList &l, int c, int q,
+                                          int k_steps, ConvItem &it) {
+  if (q < l.n_sk) {
+    const long long ut = l.lo / k_steps + q;
+    const long long s0 = ut * k_steps;
+    it.t = p.tail0 + static_cast<int>(ut);
+    it.k0 = static_cast<int>(l.lo > s0 ? l.lo - s0 : 0);
+    it.k1 = static_cast<int>(l.hi - s0 < k_steps ? l.hi - s0 : k_steps);
+    it.slot = (it.k0 == 0 && it.k1 == k_steps) ? -1 : 2 * c + q;
+    it.s0 = s0;
+    return true;
+  }
+  const long long t = static_cast<long long>(q - l.n_sk) * gridDim.x + c;
+  if (t >= l.dp_end) return false;
+  it.t = static_cast<int>(t);
+  it.k0 = 0;
+  it.k1 = k_steps;
+  it.slot = -1;
+  it.s0 = 0;
+  return true;
+}
+
+// Slot of CTA c's piece of the tail tile whose first step is s0: its first piece if its share
+// starts inside the tile, else its second.
+__device__ __forceinline__ int conv_piece_slot(const ConvParams &p, int c, long long s0) {
+  return 2 * c + (conv_sk_lo(p, c) >= s0 ? 0 : 1);
+}
+
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// A slot holds a piece as [mt][32-channel chunk][8 float4 groups][128 rows][4]: for each chunk
+// and group the 128 rows of a half are consecutive, so a warp's 32 rows move 512 contiguous bytes.
+__device__ __forceinline__ float4 *slot_group(float *slot, int mt, int cc, int v, int row) {
+  return reinterpret_cast<float4 *>(slot) + ((mt * (kBN / 32) + cc) * 8 + v) * kBM + row;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     conv3d_causal_kernel(const __grid_constant__ CUtensorMap tmx,
                          const __grid_constant__ CUtensorMap tmw, const ConvParams p) {
@@ -84,11 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain = acc_empty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *merge_word = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles = p.m_tiles * p.n_tiles;
   const int ncb = p.C_in / kBK;            // 64-channel blocks per tap
   const int k_steps = 27 * ncb;
+  const ConvList list = conv_list(p, blockIdx.x, k_steps);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -120,11 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmw);
       int n = 0;  // stage fills issued
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const ConvTile c = conv_tile(p, t);
+      ConvItem it;
+      for (int q = 0; ok && conv_item(p, list, blockIdx.x, q, k_steps, it); ++q) {
+        const ConvTile c = conv_tile(p, it.t);
         const int b = c.bt / p.T;
         const int f0 = c.bt + 2 * b;       // input frame of tap dt = 0 (streams hold T + 2)
-        for (int k = 0; k < k_steps; ++k, ++n) {
+        for (int k = it.k0; k < it.k1; ++k, ++n) {
           const int s = n % kStages;
           const uint32_t r = static_cast<uint32_t>(n / kStages);
           if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
@@ -152,13 +234,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lo0 = static_cast<uint32_t>(sdesc_sw128(smem_u32(smem), 16, 1024));
       bool ok = true;
       int n = 0, i = 0;
-      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
+      ConvItem it;
+      for (; ok && conv_item(p, list, blockIdx.x, i, k_steps, it); ++i) {
         const int acc = i & 1;
         if (!(ok = wait_bounded(&acc_empty[acc], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u, g, E)))
           break;
         tc_fence_after();
         const uint32_t d = tmem + acc * kAccCols;
-        for (int k = 0; k < k_steps; ++k, ++n) {
+        for (int k = it.k0; k < it.k1; ++k, ++n) {
           const int s = n % kStages;
           if (!(ok = wait_bounded(&full[s], static_cast<uint32_t>(n / kStages) & 1u, g, E))) break;
           tc_fence_after();
@@ -169,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int mt = 0; mt < kMT; ++mt)
               umma_ss(d + mt * kBN, f2u64(la + mt * ((kBM * kBK * 2) >> 4) + kk * 2, hi),
-                      f2u64(lb + kk * 2, hi), kId, (k > 0 || kk > 0) ? 1u : 0u);
+                      f2u64(lb + kk * 2, hi), kId, (k > it.k0 || kk > 0) ? 1u : 0u);
           umma_commit(&empty[s]);
         }
         if (ok) umma_commit(&acc_full[acc]);
@@ -184,26 +267,105 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hh = row / 16, ww = row % 16;
     bool ok = true;
     int i = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+    ConvItem it;
+    // After a timeout the four warps keep walking the same list without waiting, so that all
+    // of them reach every epi_sync (a warp that left would stall the others there).
+    for (; conv_item(p, list, blockIdx.x, i, k_steps, it); ++i) {
       const int acc = i & 1;
       if (ok)
         ok = __all_sync(kFull, wait_bounded(&acc_full[acc], static_cast<uint32_t>(i >> 1) & 1u, g, E));
-      if (!ok) break;
-      tc_fence_after();
-      const ConvTile c = conv_tile(p, t);
+      if (ok) tc_fence_after();
+      const uint32_t src0 = tmem + lane_base + acc * kAccCols;
+      // the first and last CTA holding a piece of this tile (partial pieces only)
+      int c_first = 0, c_last = 0;
+      bool merge = false;
+      if (it.slot >= 0) {
+        // a piece of a split tile: leave it in this CTA's slot, count it, merge if it was last
+        float *mine = p.slots + static_cast<long long>(it.slot) * kConvSlotFloats;
+#pragma unroll 1
+        for (int mt = 0; ok && mt < kMT; ++mt)
+#pragma unroll 1
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(src0 + mt * kBN + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              __stcg(slot_group(mine, mt, cc, v, row),
+                     make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3])));
+          }
+        __threadfence();
+        // a warp with ok false has set abort_flag before it arrives here, so row 0 counts only
+        // when all four warps hold their sums: a merge implies ok in every warp
+        epi_sync();
+        c_first = static_cast<int>(((it.s0 + 1) * p.g_sk - 1) / p.w_tail);
+        c_last = static_cast<int>(((it.s0 + k_steps) * p.g_sk - 1) / p.w_tail);
+        if (row == 0) {
+          int last = 0;
+          if (!*abort_flag) {
+            // the count word carries the launch's epoch in its high bits, so a word left by an
+            // aborted launch is never taken for a count of this one
+            unsigned *ctr = p.counters + (it.t - p.tail0);
+            const unsigned ep = p.epoch << 8;
+            unsigned old = *reinterpret_cast<volatile unsigned *>(ctr), nw;
+            while (true) {
+              nw = ((old & 0xFFFFFF00u) == ep) ? old + 1 : (ep | 1u);
+              const unsigned seen = atomicCAS(ctr, old, nw);
+              if (seen == old) break;
+              old = seen;
+            }
+            last = static_cast<int>(nw & 0xFFu) == c_last - c_first + 1;
+            if (last) atomicExch(ctr, 0u);
+          }
+          *merge_word = last;
+        }
+        epi_sync();
+        merge = *merge_word != 0;
+        epi_sync();  // merge_word is written again by the next piece
+        if (!merge) {
+          if (ok) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+          }
+          continue;
+        }
+        __threadfence();
+      }
+      if (!ok) continue;
+      const ConvTile c = conv_tile(p, it.t);
 #pragma unroll 1
       for (int mt = 0; mt < kMT; ++mt) {
       const int h = c.h0 + 8 * mt + hh, x = c.w0 + ww;
       const bool live = h < p.H && x < p.W;
       __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) +
                            ((static_cast<long long>(c.bt) * p.H + h) * p.W + x) * p.C_out;
-      const uint32_t src = tmem + lane_base + acc * kAccCols + mt * kBN;
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t o[32];
-        tmem_ld32(src + cc * 32, o);
+        tmem_ld32(src0 + mt * kBN + cc * 32, o);
         tmem_wait_ld();
         const int nb = c.n0 + cc * 32;
+        if (merge) {
+          // add the other CTAs' pieces of this tile
+#pragma unroll 1
+          for (int cp = c_first; cp <= c_last; ++cp) {
+            if (cp == static_cast<int>(blockIdx.x)) continue;
+            const float *other =
+                p.slots + static_cast<long long>(conv_piece_slot(p, cp, it.s0)) * kConvSlotFloats;
+            float4 r[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              r[v] = __ldcg(slot_group(const_cast<float *>(other), mt, cc, v, row));
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              o[4 * v] = __float_as_uint(__uint_as_float(o[4 * v]) + r[v].x);
+              o[4 * v + 1] = __float_as_uint(__uint_as_float(o[4 * v + 1]) + r[v].y);
+              o[4 * v + 2] = __float_as_uint(__uint_as_float(o[4 * v + 2]) + r[v].z);
+              o[4 * v + 3] = __float_as_uint(__uint_as_float(o[4 * v + 3]) + r[v].w);
+            }
+          }
+        }
         if (live && nb < p.C_out) {
           float bv[32];
 #pragma unroll
@@ -257,7 +419,31 @@ cudaError_t launch_conv3d_causal(const CUtensorMap &tmx, const CUtensorMap &tmw,
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  conv3d_causal_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(tmx, tmw, p);
+  ConvParams q = p;
+  q.tail0 = 0;
+  q.g_sk = 0;
+  q.w_tail = 0;
+  // stream-K over the tiles that do not fill a last whole wave, when the caller gave scratch:
+  // each tail tile is cut into at most kMaxSplit pieces (the merge reads the other pieces from
+  // L2) of at least kMinShare K steps (a piece's fp32 write-back and merge cost about as much as
+  // a few dozen steps: with 27-step tiles the split measured slower than whole tiles).  The
+  // split needs more CTAs than tail tiles, and a share is then never longer than one tile.
+  constexpr int kMaxSplit = 4;
+  constexpr long long kMinShare = 48;
+  const int tail = static_cast<int>(tiles % grid);
+  if (p.counters != nullptr && p.slots != nullptr && tiles > grid && tail > 0) {
+    const int k_steps = 27 * (p.C_in / kBK);
+    const long long w_tail = static_cast<long long>(tail) * k_steps;
+    long long g = w_tail / kMinShare;
+    if (g > static_cast<long long>(tail) * kMaxSplit) g = static_cast<long long>(tail) * kMaxSplit;
+    if (g > grid) g = grid;
+    if (g > tail) {
+      q.tail0 = static_cast<int>(tiles - tail);
+      q.g_sk = static_cast<int>(g);
+      q.w_tail = w_tail;
+    }
+  }
+  conv3d_causal_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(tmx, tmw, q);
   return cudaGetLastError();
 }
 

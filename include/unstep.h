@@ -297,13 +297,26 @@ int unstep_renoise(const void *x0, const void *eps, void *out, long long n, floa
  *                      w[o][dt][dy][dx][c] * x[b][t + dt][h + dy - 1][x + dx - 1][c],
  * positions outside the frame reading 0: output frame t sees input frames t .. t + 2.  bf16
  * tensor-core products with fp32 accumulation, output rounded to bf16 (RNE).
- * Errors: ARG (NULL pointer, size < 1), ALIGN (x, w, y not 16-byte aligned, bias not 4-byte),
- * UNSUPPORTED (C_in not a multiple of 64, C_out not a multiple of 8, sizes beyond the kernel's
- * 32-bit tile indexing), CUDA.  A device-side wait past its limit sets *dev_error.
+ *   scratch, scratch_bytes : optional (caller-allocated, caller-owned; NULL and 0 for none).
+ *          With it, the output tiles that do not fill a last whole wave of the SMs are cut
+ *          along K over all SMs (stream-K); without it they run whole, one per SM.  At least
+ *          unstep_conv3d_scratch_bytes() bytes, 16-byte aligned, ZERO-FILLED by the caller before
+ *          its first use; every call leaves it fit for the next one, including a call whose
+ *          device wait timed out.  Calls that share one scratch buffer must not run at the same
+ *          time (same stream, or ordered by events).  The result does not depend on whether
+ *          scratch is given, up to the fp32 summation order of the split tiles.
+ * Errors: ARG (NULL pointer, size < 1, scratch_bytes too small), ALIGN (x, w, y, scratch not
+ * 16-byte aligned, bias not 4-byte), UNSUPPORTED (C_in not a multiple of 64, C_out not a
+ * multiple of 8, sizes beyond the kernel's 32-bit tile indexing), CUDA.  A device-side wait past
+ * its limit sets *dev_error.
  */
 int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *y, int B, int T,
-                         int H, int W, int C_in, int C_out, int *dev_error,
-                         unstep_stream_t stream);
+                         int H, int W, int C_in, int C_out, void *scratch, size_t scratch_bytes,
+                         int *dev_error, unstep_stream_t stream);
+
+/* Bytes of unstep_conv3d_causal's optional scratch on the CURRENT device (it depends on the
+ * device's SM count, not on the shape); 0 if the device cannot be queried. */
+size_t unstep_conv3d_scratch_bytes(void);
 
 /*
  * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported

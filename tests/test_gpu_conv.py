@@ -81,3 +81,74 @@ def test_decoder_shaped_layer_on_sampled_rows():
         # is also the slice's padding at the true borders)
         want = oracle.conv3d_causal(xb[:, :, lo:hi], wb, bb)[:, :, h - lo]
         _check(got[:, :, h], xb[:, :, lo:hi], wb, bb, want, row=h - lo)
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def _counters_zero(scratch):
+    # every tail tile's count word is reset by the piece that merged it
+    return int(scratch[:4 * _sms()].view(torch.int32).abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("extra,Ci,Co", [
+    (1, 256, 128),    # one 108-step tail tile cut into 2 pieces of 54 steps
+    (37, 256, 128),   # 37 tail tiles over 83 CTAs: 48-step shares, 2-3 pieces per tile
+    (130, 128, 128),  # most of a wave: 54-step tiles over 146 CTAs, 1-2 pieces per tile
+    (30, 64, 128),    # 27-step tiles are too short to split: the scratch is left unused
+])
+def test_stream_k_tail_matches_oracle(extra, Ci, Co):
+    """Frames of one 16 x 16 tile each, SMs + extra tiles: the first wave runs whole, the extra
+    tiles are cut along K over the SMs (shares of at least 48 K steps) and merged by the last
+    piece to finish."""
+    B, T, H, Wd = 1, _sms() + extra, 16, 16
+    x, w, bias = _inputs(B, T, H, Wd, Ci, Co, seed=extra + Ci)
+    scratch = binding.conv3d_scratch()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda(), dev_error=err, scratch=scratch)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert _counters_zero(scratch)
+    xb, wb, bb = W.bits(x), W.bits(w), bias.double().numpy()
+    # the whole first wave and the tail: frames 0..3 and the last 2 + extra frames
+    for t0, t1 in ((0, 4), (T - extra - 2, T)):
+        want = oracle.conv3d_causal(xb[:, t0:t1 + 2], wb, bb)
+        _check(got[:, t0:t1].cpu().double().numpy(), xb[:, t0:t1 + 2], wb, bb, want)
+    # the split tiles differ from whole ones only in the fp32 summation order
+    whole = binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda())
+    d = (got.float() - whole.float()).abs()
+    assert float(d.max()) <= 2.0 ** -6 * float(whole.float().abs().max())
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 9, 60, 104, 128, 256),  # 504 tiles: 3 whole waves, 60 tail tiles over 67 CTAs
+    (1, 3, 60, 104, 384, 384),  # the decoder layer: 1 whole wave, 104 tail tiles in 2-3 pieces
+])
+def test_stream_k_layers_on_sampled_rows_and_repeat_calls(shape):
+    """Layer shapes with scratch: sampled rows against the oracle, the same bits on a second
+    call with the same scratch (the counters' epochs keep launches apart)."""
+    B, T, H, Wd, Ci, Co = shape
+    x, w, bias = _inputs(B, T, H, Wd, Ci, Co, seed=Ci + Co)
+    scratch = binding.conv3d_scratch()
+    xc, wc, bc = x.cuda(), w.cuda(), bias.cuda()
+    got = binding.conv3d_causal(xc, wc, bc, scratch=scratch)
+    again = binding.conv3d_causal(xc, wc, bc, scratch=scratch)
+    torch.cuda.synchronize()
+    assert _counters_zero(scratch)
+    assert torch.equal(got.view(torch.int16), again.view(torch.int16))
+    got = got.cpu().double().numpy()
+    xb, wb, bb = W.bits(x), W.bits(w), bias.double().numpy()
+    for t in (0, T - 1):
+        for h in (0, 15, 16, 59):
+            lo, hi = max(0, h - 1), min(H, h + 2)
+            want = oracle.conv3d_causal(xb[:, t:t + 3, lo:hi], wb, bb)[:, :, h - lo]
+            _check(got[:, t:t + 1, h], xb[:, t:t + 3, lo:hi], wb, bb, want, row=h - lo)
+
+
+def test_stream_k_scratch_too_small_is_rejected():
+    x, w, bias = _inputs(1, _sms() + 3, 16, 16, 64, 128, seed=3)
+    small = torch.zeros(binding.lib().unstep_conv3d_scratch_bytes() - 16, dtype=torch.uint8,
+                        device="cuda")
+    with pytest.raises(binding.UnstepError):
+        binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda(), scratch=small)

@@ -100,10 +100,11 @@ def test_conv_arguments_rejected_on_the_host():
     err = ctypes.c_void_p(0x710000)
     ok_args = (1, 3, 8, 16, 64, 128)
     f = L.unstep_conv3d_causal
-    assert f(None, p, None, p, *ok_args, err, None) == B.UNSTEP_ERR_ARG
-    assert f(p, p, None, p, *ok_args, None, None) == B.UNSTEP_ERR_ARG
-    assert f(p, p, None, p, 1, 0, 8, 16, 64, 128, err, None) == B.UNSTEP_ERR_ARG
-    assert f(odd, p, None, p, *ok_args, err, None) == B.UNSTEP_ERR_ALIGN
-    assert f(p, p, ctypes.c_void_p(0x700002), p, *ok_args, err, None) == B.UNSTEP_ERR_ALIGN
-    assert f(p, p, None, p, 1, 3, 8, 16, 48, 128, err, None) == B.UNSTEP_ERR_UNSUPPORTED
-    assert f(p, p, None, p, 1, 3, 8, 16, 64, 100, err, None) == B.UNSTEP_ERR_UNSUPPORTED
+    assert f(None, p, None, p, *ok_args, None, 0, err, None) == B.UNSTEP_ERR_ARG
+    assert f(p, p, None, p, *ok_args, None, 0, None, None) == B.UNSTEP_ERR_ARG
+    assert f(p, p, None, p, 1, 0, 8, 16, 64, 128, None, 0, err, None) == B.UNSTEP_ERR_ARG
+    assert f(odd, p, None, p, *ok_args, None, 0, err, None) == B.UNSTEP_ERR_ALIGN
+    assert f(p, p, ctypes.c_void_p(0x700002), p, *ok_args, None, 0, err, None) == B.UNSTEP_ERR_ALIGN
+    assert f(p, p, None, p, *ok_args, odd, 1 << 30, err, None) == B.UNSTEP_ERR_ALIGN
+    assert f(p, p, None, p, 1, 3, 8, 16, 48, 128, None, 0, err, None) == B.UNSTEP_ERR_UNSUPPORTED
+    assert f(p, p, None, p, 1, 3, 8, 16, 64, 100, None, 0, err, None) == B.UNSTEP_ERR_UNSUPPORTED
