@@ -624,7 +624,8 @@ int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *
     const cuuint64_t str[3] = {static_cast<cuuint64_t>(C_in) * 2,
                                static_cast<cuuint64_t>(W) * C_in * 2,
                                static_cast<cuuint64_t>(H) * W * C_in * 2};
-    const cuuint32_t box[4] = {64, 16, 8, 1};
+    // the output tile's rows and a halo row on each side, for the three dy taps at once
+    const cuuint32_t box[4] = {64, 16, static_cast<cuuint32_t>(unstep::kConvTileH + 2), 1};
     if (!encode_bf16(&tmx, x, 4, dims, str, box)) return UNSTEP_ERR_CUDA;
   }
   {

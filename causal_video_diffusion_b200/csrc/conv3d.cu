@@ -10,14 +10,16 @@
 // where each stream's input carries two history frames in front (output frame t sees input
 // frames t .. t + 2) and positions outside the frame read zero.  It is computed as an implicit
 // GEMM: M = output positions, N = output channels, K = 27 taps x C_in.  An output tile is 16
-// rows x 16 columns of one frame (two halves of 128 positions) by 128 channels; K advances 64
-// input channels of one tap at a time, and each half's A tile of that step is one TMA box {64
-// channels, 16 x, 8 y, 1 frame} of the input at the tap's offset -- it lands in shared memory as
-// 128 rows of 128 bytes with the 128-byte swizzle, exactly the K-major operand layout, and the
-// box's out-of-range part (the frame's border, the padding) is zero-filled by the TMA unit.  B is
-// the tap's {64 channels x 128 output channels} slice of the weights, shared by both halves.  The
-// pipeline is the projection GEMM's: a persistent grid, a TMA ring, tcgen05.mma M=128 N=128 K=16
-// per half into one of two TMEM accumulator sets, a 4-warp epilogue (thread = TMEM lane = output
+// rows x 16 columns of one frame (two halves of 128 positions) by 128 channels; a K step is one
+// (dt, dx) tap column and 64 input channels, all three dy taps: its A operand is one TMA box {64
+// channels, 16 x, 18 y, 1 frame} of the input (the tile's rows and one halo row on each side) at
+// the column's offset -- it lands in shared memory as 288 rows of 128 bytes with the 128-byte
+// swizzle, the K-major operand layout, and each (half, dy) operand is 128 consecutive rows of it
+// starting at a whole row of 16 positions; the box's out-of-range part (the frame's border, the
+// padding) is zero-filled by the TMA unit.  B is each tap's {64 channels x 128 output channels}
+// slice of the weights, shared by both halves.  A persistent grid, separate TMA rings for the A
+// boxes and the weight slices, tcgen05.mma M=128 N=128 K=16 per half into one of two TMEM
+// accumulator sets, a 4-warp epilogue (thread = TMEM lane = output
 // position of a half) adding the bias and storing bf16.  With caller scratch, the tiles of the
 // last, partial wave are cut along K over all SMs (stream-K, below).
 #include <cuda_bf16.h>
@@ -29,22 +31,28 @@
 namespace unstep {
 namespace {
 
-// kMT 128-position halves per output tile (rows 8 kMT x 16 columns), each its own M=128
-// product against the same weight slice, so that one B load serves kMT x 128 positions
-#ifndef UNSTEP_CONV_MT
-#define UNSTEP_CONV_MT 2
-#endif
-constexpr int kMT = UNSTEP_CONV_MT;
+// Two 128-position halves per output tile (rows 16 x 16 columns), each its own M=128 product
+// against the same weight slice, so that one B load serves 256 positions.  A K step is one
+// (dt, dx) tap column and 64 input channels: its A operand is ONE TMA box of the tile's 16 rows
+// plus a halo row above and below (18 rows x 16 columns x 64 channels), and the three dy taps
+// read it at row offsets dy, dy + 8 -- whole rows of 16 positions, i.e. multiples of 2048 bytes
+// in shared memory, so each tap's operand is the same box under a shifted descriptor.  Per K
+// step: 36 KB of A and three 16 KB weight slices for six 128x128x64 products.
+constexpr int kMT = kConvTileH / 8;
 constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kTileH = 8 * kMT, kTileW = 16;         // an output tile: 8 kMT rows x 16 columns
-constexpr int kStages = kMT == 1 ? 6 : 4;
-constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
-constexpr int kABytes = kMT * kBM * kBK * 2;         // 16 KB per 128 positions
+constexpr int kTileH = kConvTileH, kTileW = 16;      // an output tile: 16 rows x 16 columns
+constexpr int kBoxH = kTileH + 2;                    // rows of an A box: the tile and its halo
+constexpr int kRowBytes = kTileW * kBK * 2;          // one row of 16 positions x 64 channels
+constexpr int kABytes = kBoxH * kRowBytes;           // 36 KB
 constexpr int kBBytes = kBN * kBK * 2;               // 16 KB
+constexpr int kStagesA = 3, kStagesB = 7;            // A boxes and weight slices in flight
+constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
 constexpr int kAccCols = kMT * kBN;                  // TMEM columns of one accumulator set
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kSmemBar = kStages * kStageBytes;
+constexpr int kSmemB = kStagesA * kABytes;           // the weight ring follows the A ring
+constexpr int kSmemBar = kSmemB + kStagesB * kBBytes;
 constexpr int kSmemAlloc = kSmemBar + 256 + 1024;
+static_assert(kMT == 2 && kABytes % 1024 == 0 && kRowBytes % 1024 == 0, "A box layout");
+static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
@@ -157,9 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kSmemBar);
-  uint64_t *empty = full + kStages;
-  uint64_t *acc_full = empty + kStages;   // [2]
+  uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+  uint64_t *a_empty = a_full + kStagesA;
+  uint64_t *b_full = a_empty + kStagesA;
+  uint64_t *b_empty = b_full + kStagesB;
+  uint64_t *acc_full = b_empty + kStagesB;  // [2]
   uint64_t *acc_empty = acc_full + 2;     // [2]
   uint64_t *drain = acc_empty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -168,13 +178,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ncb = p.C_in / kBK;            // 64-channel blocks per tap
-  const int k_steps = 27 * ncb;
+  const int k_steps = 9 * ncb;             // (dt, dx) tap columns x channel blocks
   const ConvList list = conv_list(p, blockIdx.x, k_steps);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < kStagesA; ++s) {
+      mbar_init(&a_full[s], 1);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesB; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
@@ -199,32 +213,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmx);
       tma_prefetch_desc(&tmw);
-      int n = 0;  // stage fills issued
+      int na = 0, nb = 0;  // A boxes and weight slices issued
       bool ok = true;
       ConvItem it;
       for (int q = 0; ok && conv_item(p, list, blockIdx.x, q, k_steps, it); ++q) {
         const ConvTile c = conv_tile(p, it.t);
         const int b = c.bt / p.T;
         const int f0 = c.bt + 2 * b;       // input frame of tap dt = 0 (streams hold T + 2)
-        for (int k = it.k0; k < it.k1; ++k, ++n) {
-          const int s = n % kStages;
-          const uint32_t r = static_cast<uint32_t>(n / kStages);
-          if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
-          const int tap = k / ncb, c0 = (k - tap * ncb) * kBK;
-          const int dt = tap / 9, dy = (tap / 3) % 3, dx = tap % 3;
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          uint8_t *st = smem + s * kStageBytes;
-          // input box at the tap's offset: x and y may start at -1 (zero fill outside)
-#pragma unroll
-          for (int mt = 0; mt < kMT; ++mt)
-            tma_load_4d(st + mt * (kBM * kBK * 2), &tmx, &full[s], c0, c.w0 + dx - 1,
-                        c.h0 + 8 * mt + dy - 1, f0 + dt);
-          tma_load_3d(st + kABytes, &tmw, &full[s], c0, tap, c.n0);
+        for (int k = it.k0; ok && k < it.k1; ++k) {
+          const int col = k / ncb, c0 = (k - col * ncb) * kBK;
+          const int dt = col / 3, dx = col % 3;
+          {
+            const int s = na % kStagesA;
+            if (!(ok = wait_bounded(&a_empty[s], (static_cast<uint32_t>(na / kStagesA) & 1u) ^ 1u,
+                                    g, E)))
+              break;
+            mbar_arrive_expect_tx(&a_full[s], kABytes);
+            // rows h0 - 1 .. h0 + 16 at the tap column's offset: x and y may start at -1 and
+            // run past the frame (zero fill outside)
+            tma_load_4d(smem + s * kABytes, &tmx, &a_full[s], c0, c.w0 + dx - 1, c.h0 - 1,
+                        f0 + dt);
+            ++na;
+          }
+          for (int dy = 0; dy < 3; ++dy) {
+            const int s = nb % kStagesB;
+            if (!(ok = wait_bounded(&b_empty[s], (static_cast<uint32_t>(nb / kStagesB) & 1u) ^ 1u,
+                                    g, E)))
+              break;
+            mbar_arrive_expect_tx(&b_full[s], kBBytes);
+            tma_load_3d(smem + kSmemB + s * kBBytes, &tmw, &b_full[s], c0, dt * 9 + dy * 3 + dx,
+                        c.n0);
+            ++nb;
+          }
         }
       }
-      if (*abort_flag)
-        for (int k = max(0, n - kStages); k < n; ++k)
-          drain_wait(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
+      if (*abort_flag) {
+        for (int k = max(0, na - kStagesA); k < na; ++k)
+          drain_wait(&a_full[k % kStagesA], static_cast<uint32_t>(k / kStagesA) & 1u);
+        for (int k = max(0, nb - kStagesB); k < nb; ++k)
+          drain_wait(&b_full[k % kStagesB], static_cast<uint32_t>(k / kStagesB) & 1u);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -233,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t hi = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
       const uint32_t lo0 = static_cast<uint32_t>(sdesc_sw128(smem_u32(smem), 16, 1024));
       bool ok = true;
-      int n = 0, i = 0;
+      int na = 0, nb = 0, i = 0;
       ConvItem it;
       for (; ok && conv_item(p, list, blockIdx.x, i, k_steps, it); ++i) {
         const int acc = i & 1;
@@ -241,19 +269,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc_fence_after();
         const uint32_t d = tmem + acc * kAccCols;
-        for (int k = it.k0; k < it.k1; ++k, ++n) {
-          const int s = n % kStages;
-          if (!(ok = wait_bounded(&full[s], static_cast<uint32_t>(n / kStages) & 1u, g, E))) break;
-          tc_fence_after();
-          const uint32_t la = lo0 + static_cast<uint32_t>((s * kStageBytes) >> 4);
-          const uint32_t lb = la + static_cast<uint32_t>(kABytes >> 4);
+        for (int k = it.k0; ok && k < it.k1; ++k) {
+          const int sa = na % kStagesA;
+          if (!(ok = wait_bounded(&a_full[sa], static_cast<uint32_t>(na / kStagesA) & 1u, g, E)))
+            break;
+          const uint32_t la = lo0 + static_cast<uint32_t>((sa * kABytes) >> 4);
+          for (int dy = 0; dy < 3; ++dy) {
+            const int sb = nb % kStagesB;
+            if (!(ok = wait_bounded(&b_full[sb], static_cast<uint32_t>(nb / kStagesB) & 1u, g, E)))
+              break;
+            tc_fence_after();
+            const uint32_t lb = lo0 + static_cast<uint32_t>((kSmemB + sb * kBBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
+            for (int kk = 0; kk < kBK / 16; ++kk)
 #pragma unroll
-            for (int mt = 0; mt < kMT; ++mt)
-              umma_ss(d + mt * kBN, f2u64(la + mt * ((kBM * kBK * 2) >> 4) + kk * 2, hi),
-                      f2u64(lb + kk * 2, hi), kId, (k > it.k0 || kk > 0) ? 1u : 0u);
-          umma_commit(&empty[s]);
+              for (int mt = 0; mt < kMT; ++mt)
+                // half mt, tap dy: output row 8 mt + r reads box row 8 mt + r + dy
+                umma_ss(d + mt * kBN,
+                        f2u64(la + (((8 * mt + dy) * kRowBytes) >> 4) + kk * 2, hi),
+                        f2u64(lb + kk * 2, hi), kId,
+                        (k > it.k0 || dy > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&b_empty[sb]);
+            ++nb;
+          }
+          if (!ok) break;
+          umma_commit(&a_empty[sa]);
+          ++na;
         }
         if (ok) umma_commit(&acc_full[acc]);
       }
@@ -426,13 +467,13 @@ cudaError_t launch_conv3d_causal(const CUtensorMap &tmx, const CUtensorMap &tmw,
   // stream-K over the tiles that do not fill a last whole wave, when the caller gave scratch:
   // each tail tile is cut into at most kMaxSplit pieces (the merge reads the other pieces from
   // L2) of at least kMinShare K steps (a piece's fp32 write-back and merge cost about as much as
-  // a few dozen steps: with 27-step tiles the split measured slower than whole tiles).  The
-  // split needs more CTAs than tail tiles, and a share is then never longer than one tile.
+  // a few dozen 64-channel taps: tiles of 27 taps measured slower split than whole).  The split
+  // needs more CTAs than tail tiles, and a share is then never longer than one tile.
   constexpr int kMaxSplit = 4;
-  constexpr long long kMinShare = 48;
+  constexpr long long kMinShare = 16;  // K steps of three taps each
   const int tail = static_cast<int>(tiles % grid);
   if (p.counters != nullptr && p.slots != nullptr && tiles > grid && tail > 0) {
-    const int k_steps = 27 * (p.C_in / kBK);
+    const int k_steps = 9 * (p.C_in / kBK);
     const long long w_tail = static_cast<long long>(tail) * k_steps;
     long long g = w_tail / kMinShare;
     if (g > static_cast<long long>(tail) * kMaxSplit) g = static_cast<long long>(tail) * kMaxSplit;

@@ -153,13 +153,9 @@ struct ConvParams {
 };
 
 // Rows of a convolution output tile (two 8 x 16 halves of 128 positions).
-#ifndef UNSTEP_CONV_MT
-#define UNSTEP_CONV_MT 2
-#endif
-constexpr int kConvTileH = 8 * UNSTEP_CONV_MT;
-// One partial output tile of the conv's stream-K tail: UNSTEP_CONV_MT x 128 positions x 128
-// channels, fp32.
-constexpr long long kConvSlotFloats = UNSTEP_CONV_MT * 128ll * 128;
+constexpr int kConvTileH = 16;
+// One partial output tile of the conv's stream-K tail: 2 x 128 positions x 128 channels, fp32.
+constexpr long long kConvSlotFloats = 2 * 128ll * 128;
 // Bytes of the conv's stream-K scratch for a device with `sms` SMs: one counter per tail tile
 // (fewer tail tiles than SMs), 256-byte aligned, then 2 slots per SM.
 constexpr size_t conv_counter_bytes(int sms) {
@@ -169,8 +165,8 @@ constexpr size_t conv_scratch_bytes(int sms) {
   return conv_counter_bytes(sms) + static_cast<size_t>(2) * sms * kConvSlotFloats * 4;
 }
 
-// tmx: 4D (C_in, W, H, B*(T+2)) bf16, box (64, 16, 8, 1); tmw: 3D (C_in, 27, C_out) bf16, box
-// (64, 1, 128); both 128B swizzle.
+// tmx: 4D (C_in, W, H, B*(T+2)) bf16, box (64, 16, kConvTileH + 2, 1); tmw: 3D (C_in, 27, C_out)
+// bf16, box (64, 1, 128); both 128B swizzle.
 cudaError_t launch_conv3d_causal(const CUtensorMap &tmx, const CUtensorMap &tmw,
                                  const ConvParams &p, cudaStream_t stream);
 

@@ -93,15 +93,15 @@ def _counters_zero(scratch):
 
 
 @pytest.mark.parametrize("extra,Ci,Co", [
-    (1, 256, 128),    # one 108-step tail tile cut into 2 pieces of 54 steps
-    (37, 256, 128),   # 37 tail tiles over 83 CTAs: 48-step shares, 2-3 pieces per tile
-    (130, 128, 128),  # most of a wave: 54-step tiles over 146 CTAs, 1-2 pieces per tile
-    (30, 64, 128),    # 27-step tiles are too short to split: the scratch is left unused
+    (1, 256, 128),    # one 36-step tail tile cut into 2 pieces of 18 steps
+    (37, 256, 128),   # 37 tail tiles over 83 CTAs: 16-step shares, 2-3 pieces per tile
+    (130, 128, 128),  # most of a wave: 18-step tiles over 146 CTAs, 1-2 pieces per tile
+    (30, 64, 128),    # 9-step tiles are too short to split: the scratch is left unused
 ])
 def test_stream_k_tail_matches_oracle(extra, Ci, Co):
     """Frames of one 16 x 16 tile each, SMs + extra tiles: the first wave runs whole, the extra
-    tiles are cut along K over the SMs (shares of at least 48 K steps) and merged by the last
-    piece to finish."""
+    tiles are cut along K over the SMs (shares of at least 16 K steps of three 64-channel taps)
+    and merged by the last piece to finish."""
     B, T, H, Wd = 1, _sms() + extra, 16, 16
     x, w, bias = _inputs(B, T, H, Wd, Ci, Co, seed=extra + Ci)
     scratch = binding.conv3d_scratch()
