@@ -73,9 +73,9 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-ATTN_SOURCES = ("window_attn.cu", "sm100.cuh", "internal.h")
-GEMM_SOURCES = ("gemm2sm.cu", "sm100.cuh", "internal.h")
-CONV_SOURCES = ("conv3d.cu", "sm100.cuh", "internal.h")
+ATTN_SOURCES = ("window_attn.cu", "sm100.cuh", "internal.h", "limits.h")
+GEMM_SOURCES = ("gemm2sm.cu", "sm100.cuh", "gemm.h", "limits.h")
+CONV_SOURCES = ("conv3d.cu", "sm100.cuh", "conv3d.h", "limits.h")
 
 
 def source_digest(names=ATTN_SOURCES) -> str:

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libunstep.so")
 SOURCES = ["api.cu", "rope_append.cu", "window_attn.cu", "lowrank_gemm.cu", "renoise.cu",
            "conv3d.cu", "gemm2sm.cu"]
-HEADERS = ["internal.h", "sm100.cuh"]
+HEADERS = ["internal.h", "limits.h", "gemm.h", "conv3d.h", "sm100.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",

@@ -15,6 +15,8 @@
 #include <cuda_runtime.h>
 
 #include "../../include/unstep.h"
+#include "conv3d.h"
+#include "gemm.h"
 #include "internal.h"
 
 namespace {

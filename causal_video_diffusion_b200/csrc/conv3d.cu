@@ -25,7 +25,7 @@
 #include <cuda_bf16.h>
 
 #include "../../include/unstep.h"
-#include "internal.h"
+#include "conv3d.h"
 #include "sm100.cuh"
 
 namespace unstep {
@@ -45,7 +45,14 @@ constexpr int kBoxH = kTileH + 2;                    // rows of an A box: the ti
 constexpr int kRowBytes = kTileW * kBK * 2;          // one row of 16 positions x 64 channels
 constexpr int kABytes = kBoxH * kRowBytes;           // 36 KB
 constexpr int kBBytes = kBN * kBK * 2;               // 16 KB
-constexpr int kStagesA = 3, kStagesB = 7;            // A boxes and weight slices in flight
+#ifndef UNSTEP_CONV_STAGES_A
+#define UNSTEP_CONV_STAGES_A 3
+#endif
+#ifndef UNSTEP_CONV_STAGES_B
+#define UNSTEP_CONV_STAGES_B 6
+#endif
+constexpr int kStagesA = UNSTEP_CONV_STAGES_A;       // A boxes in flight
+constexpr int kStagesB = UNSTEP_CONV_STAGES_B;       // weight slices in flight
 constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
 constexpr int kAccCols = kMT * kBN;                  // TMEM columns of one accumulator set
 constexpr int kSmemB = kStagesA * kABytes;           // the weight ring follows the A ring

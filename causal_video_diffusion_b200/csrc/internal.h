@@ -1,14 +1,14 @@
-// internal.h -- launch parameters shared between the host API (api.cu) and the kernels.
+// internal.h -- launch parameters of the RoPE/append, attention and renoise kernels, shared
+// between the host API (api.cu) and those kernels.
 #pragma once
 
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-namespace unstep {
+#include "limits.h"
 
-// Default limit of every device-side wait: no legitimate wait of these kernels lasts this long.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+namespace unstep {
 
 // Division by a run-time invariant d by multiply-high (Granlund & Montgomery, "Division by
 // invariant integers using multiplication", PLDI 1994): with l = ceil(log2 d) and
@@ -123,52 +123,6 @@ cudaError_t launch_window_attn(int D, const CUtensorMap &tmap_q, const CUtensorM
                                cudaStream_t stream);
 
 cudaError_t launch_wait_timeout_selftest(int *dev_error, uint64_t limit_ns, cudaStream_t stream);
-
-// C[M][N] (ldc) = A[M][K] * B[N][K]^T, bf16, fp32 accumulation; tma: 2D (K, M) box (64, 128),
-// tmb: 2D (K, N) box (64, 128), both 128B swizzle.
-cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
-                                int N, int K, int ldc, int *dev_error, cudaStream_t stream);
-
-// The same product on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles); same tensor maps.
-cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
-                                   int N, int K, int ldc, int *dev_error, cudaStream_t stream);
-
-// Causal 3x3x3 convolution (channels-last implicit GEMM); see unstep_conv3d_causal.
-struct ConvParams {
-  void *y;            // bf16 [B][T][H][W][C_out]
-  const float *bias;  // [C_out] or null
-  int *dev_error;
-  uint64_t wait_limit_ns;
-  int B, T, H, W, C_in, C_out;
-  int tiles_h, tiles_w;   // output tiles of kConvTileH rows x 16 columns per frame
-  int m_tiles, n_tiles;   // B*T*tiles_h*tiles_w position tiles; ceil(C_out / 128) channel tiles
-  // stream-K tail (g_sk = 0: none, every tile whole).  Tiles [0, tail0) are taken whole, tile
-  // w*grid + c by CTA c; the K steps of tiles [tail0, m_tiles*n_tiles) are cut evenly over
-  // g_sk CTAs, w_tail steps in all.
-  int tail0, g_sk;
-  long long w_tail;
-  unsigned *counters;     // one word per tail tile: epoch << 8 | pieces counted
-  float *slots;           // 2 g_sk slots of kConvSlotFloats fp32 partial sums
-  unsigned epoch;         // 1 .. 2^24 - 1, different for each launch
-};
-
-// Rows of a convolution output tile (two 8 x 16 halves of 128 positions).
-constexpr int kConvTileH = 16;
-// One partial output tile of the conv's stream-K tail: 2 x 128 positions x 128 channels, fp32.
-constexpr long long kConvSlotFloats = 2 * 128ll * 128;
-// Bytes of the conv's stream-K scratch for a device with `sms` SMs: one counter per tail tile
-// (fewer tail tiles than SMs), 256-byte aligned, then 2 slots per SM.
-constexpr size_t conv_counter_bytes(int sms) {
-  return (static_cast<size_t>(sms) * 4 + 255) / 256 * 256;
-}
-constexpr size_t conv_scratch_bytes(int sms) {
-  return conv_counter_bytes(sms) + static_cast<size_t>(2) * sms * kConvSlotFloats * 4;
-}
-
-// tmx: 4D (C_in, W, H, B*(T+2)) bf16, box (64, 16, kConvTileH + 2, 1); tmw: 3D (C_in, 27, C_out)
-// bf16, box (64, 1, 128); both 128B swizzle.
-cudaError_t launch_conv3d_causal(const CUtensorMap &tmx, const CUtensorMap &tmw,
-                                 const ConvParams &p, cudaStream_t stream);
 
 // out[i] = (1 - sigma) * x0[i] + sigma * eps[i], bf16, n elements.
 cudaError_t launch_renoise(const void *x0, const void *eps, void *out, long long n, float sigma,

@@ -13,7 +13,7 @@
 #include <cuda_bf16.h>
 
 #include "../../include/unstep.h"
-#include "internal.h"
+#include "gemm.h"
 #include "sm100.cuh"
 
 namespace unstep {
