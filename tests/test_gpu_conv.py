@@ -152,3 +152,22 @@ def test_stream_k_scratch_too_small_is_rejected():
                         device="cuda")
     with pytest.raises(binding.UnstepError):
         binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda(), scratch=small)
+
+
+def test_stream_k_with_ragged_tiles_and_two_streams():
+    """Split tiles at the ragged edges: 13 x 21 frames (8 + 5 rows of a 16-row tile, 16 + 5
+    columns), C_out = 200 (a 72-channel tile), B = 2; the tail is cut over the SMs."""
+    B, H, Wd, Ci, Co = 2, 13, 21, 256, 200
+    # 2 position tiles per frame x 2 channel tiles; frames per stream so that the tile count is
+    # SMs + 40 (rounded up to whole frames of both streams)
+    T = -(-(_sms() + 40) // (B * 2 * 2))
+    x, w, bias = _inputs(B, T, H, Wd, Ci, Co, seed=13)
+    scratch = binding.conv3d_scratch()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda(), dev_error=err, scratch=scratch)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert _counters_zero(scratch)
+    xb, wb, bb = W.bits(x), W.bits(w), bias.double().numpy()
+    want = oracle.conv3d_causal(xb, wb, bb)
+    _check(got.cpu().double().numpy(), xb, wb, bb, want)
