@@ -17,11 +17,11 @@
 // swizzle, the K-major operand layout, and each (half, dy) operand is 128 consecutive rows of it
 // starting at a whole row of 16 positions; the box's out-of-range part (the frame's border, the
 // padding) is zero-filled by the TMA unit.  B is each tap's {64 channels x 128 output channels}
-// slice of the weights, shared by both halves.  A persistent grid, separate TMA rings for the A
-// boxes and the weight slices, tcgen05.mma M=128 N=128 K=16 per half into one of two TMEM
-// accumulator sets, a 4-warp epilogue (thread = TMEM lane = output
-// position of a half) adding the bias and storing bf16.  With caller scratch, the tiles of the
-// last, partial wave are cut along K over all SMs (stream-K, below).
+// slice of the weights, shared by both halves.  A persistent grid, a TMA ring of two 84 KB
+// stages (a step's A box and weight slices), tcgen05.mma M=128 N=128 K=16 per half into one of
+// two TMEM accumulator sets, a 4-warp epilogue (thread = TMEM lane = output position of a half)
+// adding the bias and storing bf16.  With caller scratch, the tiles of the last, partial wave are
+// cut along K over all SMs (stream-K, below).
 #include <cuda_bf16.h>
 
 #include "../../include/unstep.h"
@@ -45,20 +45,18 @@ constexpr int kBoxH = kTileH + 2;                    // rows of an A box: the ti
 constexpr int kRowBytes = kTileW * kBK * 2;          // one row of 16 positions x 64 channels
 constexpr int kABytes = kBoxH * kRowBytes;           // 36 KB
 constexpr int kBBytes = kBN * kBK * 2;               // 16 KB
-#ifndef UNSTEP_CONV_STAGES_A
-#define UNSTEP_CONV_STAGES_A 3
-#endif
-#ifndef UNSTEP_CONV_STAGES_B
-#define UNSTEP_CONV_STAGES_B 6
-#endif
-constexpr int kStagesA = UNSTEP_CONV_STAGES_A;       // A boxes in flight
-constexpr int kStagesB = UNSTEP_CONV_STAGES_B;       // weight slices in flight
+// One stage = one K step: the A box and the step's three weight slices under ONE barrier, so
+// that the MMA thread waits once and commits once per 24 products.  A barrier per weight slice
+// was 12-15 % slower and separate A and weight rings 2-4 % slower, with deeper rings no faster:
+// the synchronisation points per step, not the lookahead, limited the MMA issue.
+constexpr int kStageBytes = kABytes + 3 * kBBytes;   // 84 KB
+constexpr int kStages = 2;
 constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
 constexpr int kAccCols = kMT * kBN;                  // TMEM columns of one accumulator set
-constexpr int kSmemB = kStagesA * kABytes;           // the weight ring follows the A ring
-constexpr int kSmemBar = kSmemB + kStagesB * kBBytes;
+constexpr int kSmemBar = kStages * kStageBytes;
 constexpr int kSmemAlloc = kSmemBar + 256 + 1024;
-static_assert(kMT == 2 && kABytes % 1024 == 0 && kRowBytes % 1024 == 0, "A box layout");
+static_assert(kMT == 2 && kABytes % 1024 == 0 && kRowBytes % 1024 == 0 &&
+                  kStageBytes % 1024 == 0, "stage layout");
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
@@ -172,11 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + kSmemBar);
-  uint64_t *a_empty = a_full + kStagesA;
-  uint64_t *b_full = a_empty + kStagesA;
-  uint64_t *b_empty = b_full + kStagesB;
-  uint64_t *acc_full = b_empty + kStagesB;  // [2]
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;   // [2]
   uint64_t *acc_empty = acc_full + 2;     // [2]
   uint64_t *drain = acc_empty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -189,13 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const ConvList list = conv_list(p, blockIdx.x, k_steps);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStagesA; ++s) {
-      mbar_init(&a_full[s], 1);
-      mbar_init(&a_empty[s], 1);
-    }
-    for (int s = 0; s < kStagesB; ++s) {
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
@@ -220,46 +212,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmx);
       tma_prefetch_desc(&tmw);
-      int na = 0, nb = 0;  // A boxes and weight slices issued
+      int n = 0;  // stages filled
       bool ok = true;
       ConvItem it;
       for (int q = 0; ok && conv_item(p, list, blockIdx.x, q, k_steps, it); ++q) {
         const ConvTile c = conv_tile(p, it.t);
         const int b = c.bt / p.T;
         const int f0 = c.bt + 2 * b;       // input frame of tap dt = 0 (streams hold T + 2)
-        for (int k = it.k0; ok && k < it.k1; ++k) {
+        for (int k = it.k0; k < it.k1; ++k, ++n) {
           const int col = k / ncb, c0 = (k - col * ncb) * kBK;
           const int dt = col / 3, dx = col % 3;
-          {
-            const int s = na % kStagesA;
-            if (!(ok = wait_bounded(&a_empty[s], (static_cast<uint32_t>(na / kStagesA) & 1u) ^ 1u,
-                                    g, E)))
-              break;
-            mbar_arrive_expect_tx(&a_full[s], kABytes);
-            // rows h0 - 1 .. h0 + 16 at the tap column's offset: x and y may start at -1 and
-            // run past the frame (zero fill outside)
-            tma_load_4d(smem + s * kABytes, &tmx, &a_full[s], c0, c.w0 + dx - 1, c.h0 - 1,
-                        f0 + dt);
-            ++na;
-          }
-          for (int dy = 0; dy < 3; ++dy) {
-            const int s = nb % kStagesB;
-            if (!(ok = wait_bounded(&b_empty[s], (static_cast<uint32_t>(nb / kStagesB) & 1u) ^ 1u,
-                                    g, E)))
-              break;
-            mbar_arrive_expect_tx(&b_full[s], kBBytes);
-            tma_load_3d(smem + kSmemB + s * kBBytes, &tmw, &b_full[s], c0, dt * 9 + dy * 3 + dx,
+          const int s = n % kStages;
+          if (!(ok = wait_bounded(&empty[s], (static_cast<uint32_t>(n / kStages) & 1u) ^ 1u, g, E)))
+            break;
+          uint8_t *st = smem + s * kStageBytes;
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          // rows h0 - 1 .. h0 + 16 at the tap column's offset: x and y may start at -1 and run
+          // past the frame (zero fill outside)
+          tma_load_4d(st, &tmx, &full[s], c0, c.w0 + dx - 1, c.h0 - 1, f0 + dt);
+          for (int dy = 0; dy < 3; ++dy)
+            tma_load_3d(st + kABytes + dy * kBBytes, &tmw, &full[s], c0, dt * 9 + dy * 3 + dx,
                         c.n0);
-            ++nb;
-          }
         }
       }
-      if (*abort_flag) {
-        for (int k = max(0, na - kStagesA); k < na; ++k)
-          drain_wait(&a_full[k % kStagesA], static_cast<uint32_t>(k / kStagesA) & 1u);
-        for (int k = max(0, nb - kStagesB); k < nb; ++k)
-          drain_wait(&b_full[k % kStagesB], static_cast<uint32_t>(k / kStagesB) & 1u);
-      }
+      if (*abort_flag)
+        for (int k = max(0, n - kStages); k < n; ++k)
+          drain_wait(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -268,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t hi = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
       const uint32_t lo0 = static_cast<uint32_t>(sdesc_sw128(smem_u32(smem), 16, 1024));
       bool ok = true;
-      int na = 0, nb = 0, i = 0;
+      int n = 0, i = 0;
       ConvItem it;
       for (; ok && conv_item(p, list, blockIdx.x, i, k_steps, it); ++i) {
         const int acc = i & 1;
@@ -276,17 +254,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc_fence_after();
         const uint32_t d = tmem + acc * kAccCols;
-        for (int k = it.k0; ok && k < it.k1; ++k) {
-          const int sa = na % kStagesA;
-          if (!(ok = wait_bounded(&a_full[sa], static_cast<uint32_t>(na / kStagesA) & 1u, g, E)))
-            break;
-          const uint32_t la = lo0 + static_cast<uint32_t>((sa * kABytes) >> 4);
+        for (int k = it.k0; k < it.k1; ++k, ++n) {
+          const int s = n % kStages;
+          if (!(ok = wait_bounded(&full[s], static_cast<uint32_t>(n / kStages) & 1u, g, E))) break;
+          tc_fence_after();
+          const uint32_t la = lo0 + static_cast<uint32_t>((s * kStageBytes) >> 4);
+#pragma unroll
           for (int dy = 0; dy < 3; ++dy) {
-            const int sb = nb % kStagesB;
-            if (!(ok = wait_bounded(&b_full[sb], static_cast<uint32_t>(nb / kStagesB) & 1u, g, E)))
-              break;
-            tc_fence_after();
-            const uint32_t lb = lo0 + static_cast<uint32_t>((kSmemB + sb * kBBytes) >> 4);
+            const uint32_t lb = la + static_cast<uint32_t>((kABytes + dy * kBBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk)
 #pragma unroll
@@ -296,12 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         f2u64(la + (((8 * mt + dy) * kRowBytes) >> 4) + kk * 2, hi),
                         f2u64(lb + kk * 2, hi), kId,
                         (k > it.k0 || dy > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(&b_empty[sb]);
-            ++nb;
           }
-          if (!ok) break;
-          umma_commit(&a_empty[sa]);
-          ++na;
+          umma_commit(&empty[s]);
         }
         if (ok) umma_commit(&acc_full[acc]);
       }
