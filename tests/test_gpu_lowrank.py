@@ -21,7 +21,9 @@ def _rel_errors(got, want):
                                    (257, 520, 72), (129, 264, 200),
                                    # 3-4 tiles per persistent pair / CTA: both accumulator sets
                                    # of each go through both barrier phases
-                                   (4096, 4096, 128), (65536, 200, 64)])
+                                   (4096, 4096, 128), (65536, 200, 64),
+                                   # CTA pairs with K ending inside a 128- and a 192-deep step
+                                   (512, 512, 200), (300, 264, 1416)])
 def test_gemm_matches_oracle(M, N, K):
     a = W.gen_act(M * 7 + 1, M, K)
     b = W.gen_act(N * 11 + 2, N, K)
