@@ -582,7 +582,7 @@ def run_vae_conv(args, rank, local_rank, world):
                                f"C_out={C}, channels-last", "l2": "flushed between steps"},
         "scaling": "weak", "vs_baseline": None,
         "gpu_launches": args.steps,
-        "roofline": {"kernel": "conv3d_causal_kernel", "bound": "tensor", "achieved": round(tf, 2),
+        "roofline": {"kernel": "conv3d_causal_pair_kernel", "bound": "tensor", "achieved": round(tf, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": src,
                      "flops_per_launch": flops,

@@ -635,7 +635,7 @@ int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *
                                 static_cast<cuuint64_t>(C_out)};
     const cuuint64_t str[2] = {static_cast<cuuint64_t>(C_in) * 2,
                                static_cast<cuuint64_t>(C_in) * 27 * 2};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(unstep::conv_weight_box_n(H))};
     if (!encode_bf16(&tmw, w, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
   }
   unstep::ConvParams p{};

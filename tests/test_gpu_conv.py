@@ -171,3 +171,28 @@ def test_stream_k_with_ragged_tiles_and_two_streams():
     xb, wb, bb = W.bits(x), W.bits(w), bias.double().numpy()
     want = oracle.conv3d_causal(xb, wb, bb)
     _check(got.cpu().double().numpy(), xb, wb, bb, want)
+
+
+def test_pair_tiles_with_stream_k_at_ragged_edges():
+    """Frames taller than one tile run on CTA pairs (32-row tiles, each CTA 16 rows and half of
+    every weight slice).  H = 40: the second pair row has 8 live rows in its first CTA and none
+    in its second; W = 21 (16 + 5 columns), C_out = 200 (a 72-channel tile, so the second CTA's
+    weight half is partly and then wholly past C_out), B = 2, and tiles beyond the last whole wave
+    of pairs cut along K, against the full oracle."""
+    B, H, Wd, Ci, Co = 2, 40, 21, 128, 200
+    pairs = _sms() // 2
+    # 2 pair rows x 2 column tiles x 2 channel tiles per frame; about 30 tail tiles
+    T = -(-(pairs + 30) // (B * 8))
+    x, w, bias = _inputs(B, T, H, Wd, Ci, Co, seed=40)
+    scratch = binding.conv3d_scratch()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda(), dev_error=err, scratch=scratch)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert _counters_zero(scratch)
+    xb, wb, bb = W.bits(x), W.bits(w), bias.double().numpy()
+    want = oracle.conv3d_causal(xb, wb, bb)
+    _check(got.cpu().double().numpy(), xb, wb, bb, want)
+    whole = binding.conv3d_causal(x.cuda(), w.cuda(), bias.cuda())
+    d = (got.float() - whole.float()).abs()
+    assert float(d.max()) <= 2.0 ** -6 * float(whole.float().abs().max())
