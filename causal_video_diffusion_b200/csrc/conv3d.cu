@@ -96,10 +96,10 @@ __device__ __forceinline__ ConvTile conv_tile(const ConvParams &p, int t, uint32
 }
 
 // ---------------------------------------------------------------------------------------------
-// Work list of unit c (a CTA, or a CTA pair, which walks one list).  The grid is persistent.
-// Without a stream-K tail (g_sk = 0) unit c takes tiles c, c + units, ... whole.  With one, it first takes its share [lo, hi) of the tail tiles'
-// K steps (at most two pieces, as a share is never longer than one tile), then whole tiles
-// w*grid + c below tail0.  The tail comes first so that the merges of split tiles overlap the
+// Work list of unit c (a CTA, or a CTA pair walking one list); the grid is persistent.  Without
+// a stream-K tail (g_sk = 0) unit c takes tiles c, c + units, ... whole.  With one, it first takes
+// its share [lo, hi) of the tail tiles' K steps (at most two pieces, as a share is never longer
+// than one tile), then whole tiles w*units + c below tail0.  The tail comes first so that the merges of split tiles overlap the
 // whole tiles' main loops instead of ending the launch.  A piece that is not a whole tile leaves
 // its fp32 sums in the CTA's slot 2 (kCta c + rank) + (piece index); the last of a tile's pieces
 // to finish (an atomic count per tile and rank) adds the others' slots to its own accumulator and
@@ -434,7 +434,7 @@ __device__ __forceinline__ void conv_body(const CUtensorMap &tmx, const CUtensor
         ok = __all_sync(kFull, wait_bounded(&acc_full[acc], static_cast<uint32_t>(i >> 1) & 1u, g, E));
       if (ok) tc_fence_after();
       const uint32_t src0 = tmem + lane_base + acc * kAccCols;
-      // the first and last CTA holding a piece of this tile (partial pieces only)
+      // the first and last unit holding a piece of this tile (partial pieces only)
       int c_first = 0, c_last = 0;
       bool merge = false;
       if (it.slot >= 0) {
@@ -502,7 +502,7 @@ __device__ __forceinline__ void conv_body(const CUtensorMap &tmx, const CUtensor
         tmem_wait_ld();
         const int nb = c.n0 + cc * 32;
         if (merge) {
-          // add the other CTAs' pieces of this tile
+          // add the other units' pieces of this tile (this CTA's rank)
 #pragma unroll 1
           for (int cp = c_first; cp <= c_last; ++cp) {
             if (cp == unit) continue;
