@@ -1,8 +1,8 @@
 // api.cu -- host side of the C ABI declared in include/unstep.h: argument validation, cache
 // metadata, the RoPE coefficient tables, window resolution, TMA descriptors and launches.
 //
-// UnStep paper (arXiv 2609.32518), abstract: RoPE "with cached coefficients", KV indexing and a
-// limited temporal window of the attention KV cache; Table 3: chunks of three latent frames.
+// UnStep paper (arXiv 2609.32518), abstract: RoPE from precomputed coefficients, KV indexing and
+// a limited temporal window of the attention KV cache; Table 3: chunks of three latent frames.
 #include <atomic>
 #include <cmath>
 #include <cstdlib>

@@ -286,8 +286,8 @@ int unstep_renoise(const void *x0, const void *eps, void *out, long long n, floa
                    unstep_stream_t stream);
 
 /*
- * Causal 3x3x3 convolution of a video VAE decoder, channels-last (the abstract's "VAE decoding
- * with optimized memory layout, precision, and convolution kernels"; Table 1 row C2).
+ * Causal 3x3x3 convolution of a video VAE decoder, channels-last (abstract and Table 1 row C2:
+ * the decoder is sped up through its memory layout, precision and convolution kernels).
  *   x    : bf16 [B][T + 2][H][W][C_in]; each stream's first two frames are its causal history
  *          (the last two input frames of the previous chunk, or zeros at the stream's start).
  *   w    : bf16 [C_out][3][3][3][C_in], taps (dt, dy, dx).

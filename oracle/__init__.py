@@ -6,7 +6,7 @@ TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the CP
 What it computes follows "UnStep: Training-Free Acceleration of Causal Video Diffusion with Fewer
 Steps Than Distillation" (arXiv 2609.32518): the abstract's runtime stack (RoPE with cached
 coefficients, KV indexing, a temporal window limit on the attention KV cache) and Table 1 row C4
-("+ limited attention window").  The pages print no formulas, so the oracle writes out the
+(the attention window limit added).  The pages print no formulas, so the oracle writes out the
 textbook definitions:
 
 * ``rope3d`` -- 3D rotary embedding, channel blocks (t, h, w) of widths (d_t, d_h, d_w), adjacent
@@ -355,8 +355,8 @@ def renoise(x0_bits: np.ndarray, eps_bits: np.ndarray, sigma: float) -> np.ndarr
 
 
 # --------------------------------------------------------------------------------------------
-# Causal 3D convolution of the VAE decoder (abstract: "VAE decoding with optimized memory layout,
-# precision, and convolution kernels"; Table 1 row C2)
+# Causal 3D convolution of the VAE decoder (abstract and Table 1 row C2: the decoder is sped up
+# through its memory layout, precision and convolution kernels)
 # --------------------------------------------------------------------------------------------
 
 def conv3d_causal(x_bits: np.ndarray, w_bits: np.ndarray,

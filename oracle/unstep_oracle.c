@@ -8,7 +8,7 @@
  * Source: "UnStep: Training-Free Acceleration of Causal Video Diffusion with Fewer Steps Than
  * Distillation" (arXiv 2609.32518), abstract: the DiT runtime stack applies RoPE from cached
  * coefficients, indexes a KV cache, and limits the temporal window that the attention KV cache
- * retains; Table 1 row C4 ("+ limited attention window").  The pages give no formulas for these
+ * retains; Table 1 row C4 (the attention window limit added).  The pages give no formulas for these
  * steps, so this file writes out the textbook definitions they name:
  *
  *   3D RoPE: the head dimension D is split into a temporal, a height and a width block
