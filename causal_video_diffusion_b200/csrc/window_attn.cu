@@ -7,7 +7,7 @@
 //
 //   S_j  = Q K_j^T                      tcgen05.mma, A = Q (smem), B = K_j (smem), fp32 in TMEM
 //   m    = running max (raised lazily), P_j = exp2(S_j * log2(e)/sqrt(D) - m)   (fp32 -> bf16)
-//   O   += P_j V_j                      tcgen05.mma, A = P_j (TMEM, aliasing S_j), B = V_j (smem)
+//   O   += P_j V_j                      tcgen05.mma, A = P_j (TMEM), B = V_j (smem)
 //   l   += rowsum(P_j);   out = O / l  (bf16)
 //
 // Work split of one CTA (one (stream, head) and two 128-row query tiles, 384 threads):
@@ -20,7 +20,8 @@
 // When q arrives un-rotated, each softmax warpgroup first applies the 3D RoPE to its loaded Q
 // tile in shared memory (once per segment, from coefficient rows staged in shared memory),
 // before the MMA issuer may use it.
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D); P0 and P1
+// alias S0 and S1 for D = 128 and sit at [384,448) and [448,512) for D = 64.
 //
 // The ring cache holds the window as at most two contiguous row ranges; each range is tiled on
 // its own (its last tile masked), so a tile never straddles the wrap and the ring slot offset is
@@ -76,6 +77,13 @@ struct Cfg {
   static constexpr int kSmemAlloc = (kSmemUsed + 1024 > 118 * 1024) ? kSmemUsed + 1024
                                                                     : 118 * 1024;
   static constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO0 = 256, kTmO1 = 256 + D;
+  // P (bf16, 64 columns per tile).  tcgen05.mma operations are only guaranteed to execute in
+  // issue order when they have the same shape; QK^T (N = 128) may overwrite the S columns
+  // while the previous PV (N = D) still reads them unless N = D.  So P aliases S only for
+  // D = 128; for D = 64 it has columns of its own (the commit that announces the next S also
+  // covers the previous PV, so P is never rewritten while a PV reads it).
+  static constexpr uint32_t kTmP0 = D == 128 ? kTmS0 : 384, kTmP1 = D == 128 ? kTmS1 : 448;
+  static_assert(D == 128 || 256 + 2 * D <= 384, "TMEM columns");
   static constexpr uint32_t kTmCols = 512;
 };
 
@@ -125,8 +133,8 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
 }
 
 // P for one 32-column chunk of a row: p = 2^(s * scale - m), summed into acc (four packed
-// accumulators), rounded to bf16 pairs and stored to the 16 TMEM columns at `taddr` (the P
-// columns alias the S columns already read).  kMasked: columns >= valid are zero (a segment's
+// accumulators), rounded to bf16 pairs and stored to the 16 TMEM columns at `taddr` (for
+// D = 128 the P columns alias the S columns already read).  kMasked: columns >= valid are zero (a segment's
 // last, partial tile), all exponentials on MUFU so that masked ones are exactly 0.
 template <bool kMasked>
 __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], int col0, int valid,
@@ -563,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto pv = [&](int t, int s, bool acc) {
           const uint32_t dO = tmem + (t ? C::kTmO1 : C::kTmO0);
-          const uint32_t aP = tmem + (t ? C::kTmS1 : C::kTmS0);
+          const uint32_t aP = tmem + (t ? C::kTmP1 : C::kTmP0);
           const uint32_t vb = loV + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -640,6 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = threadIdx.x & 127;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base + (i ? C::kTmS1 : C::kTmS0);
+    const uint32_t tP = tmem + lane_base + (i ? C::kTmP1 : C::kTmP0);
     const uint32_t tO = tmem + lane_base + (i ? C::kTmO1 : C::kTmO0);
     const float scale = p.scale_log2;
     constexpr int kTileFloats = D * 128 + 256;  // one query tile of a scratch slot
@@ -734,11 +743,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!masked) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            exp_chunk<false>(s[c], c * 32, 128, sc2, nm2, acc, tS + c * 16);
+            exp_chunk<false>(s[c], c * 32, 128, sc2, nm2, acc, tP + c * 16);
         } else {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            exp_chunk<true>(s[c], c * 32, valid, sc2, nm2, acc, tS + c * 16);
+            exp_chunk<true>(s[c], c * 32, valid, sc2, nm2, acc, tP + c * 16);
         }
         float a0, a1;
         f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
