@@ -74,6 +74,7 @@ def load_peaks():
 
 
 ATTN_SOURCES = ("window_attn.cu", "sm100.cuh", "internal.h", "limits.h")
+ROPE_SOURCES = ("rope_append.cu", "internal.h", "limits.h")
 GEMM_SOURCES = ("gemm2sm.cu", "sm100.cuh", "gemm.h", "limits.h")
 CONV_SOURCES = ("conv3d.cu", "sm100.cuh", "conv3d.h", "limits.h")
 
@@ -169,6 +170,27 @@ class ClockSampler:
 # the CUDA arm
 # ----------------------------------------------------------------------------------------------
 
+def arm_config(wl, world, args):
+    """The ``config`` object of a bench line, identical for the CUDA arm and the reference arm."""
+    s = wl.shape
+    Lk = wl.keys_for_chunk(wl.chunks - 1)
+    fq = args.q_rope == "attn"
+    strong = args.scaling == "strong"
+    return {
+        "workload": f"{wl.name}: B={s.B} H={s.H} D={s.D} grid={s.Hg}x{s.Wg} "
+                    f"L={s.L} keys={Lk} window={wl.window} cap={wl.cap}",
+        "per_rank": ("a (stream, head) shard of the workload, streams first, then heads"
+                     if strong else "one independent copy of the workload per GPU")
+        if world > 1 else "the whole workload",
+        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, then "
+              f"{L2_FLUSH_BYTES >> 20} MiB read)",
+        "parallelism": (f"(stream, head) shards x{world}" if strong else
+                        f"independent streams x{world}"),
+        "q_rope": "in the attention prologue (append moves k, v only)" if fq else
+                  "in the append (q rotated in place)",
+    }
+
+
 def run_ours(args, rank, local_rank, world):
     import torch
     from causal_video_diffusion_b200 import binding
@@ -184,15 +206,28 @@ def run_ours(args, rank, local_rank, world):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     stream = torch.cuda.current_stream()
-    seed = rank_seed(args.seed, rank)
     last = wl.chunks - 1
     F = s.chunk_frames
     f_last = wl.frame_idx(last)
     Lk = wl.keys_for_chunk(last)
-    flops = wl.attn_flops(last)
+    strong = args.scaling == "strong" and world > 1
+    if strong:
+        # one workload split over the ranks: every rank draws the same activations and works on
+        # its (stream, head) shard of them, in place; no collective touches the data
+        from causal_video_diffusion_b200 import shard as S
+        sh = S.plan(s.B, s.H, world)[rank]
+        seed = args.seed
+    else:
+        # weak scaling: every rank streams its own copy of the workload (its own seed)
+        sh = None
+        seed = rank_seed(args.seed, rank)
+    nb, nh = (sh.nb, sh.nh) if strong else (s.B, s.H)
+    flops = wl.attn_flops(last)                          # the workload (one rank's, if weak)
+    flops_rank = 4 * nb * nh * s.L * Lk * s.D            # what this rank's launches compute
 
-    cache = binding.LayerCache(s.B, s.H, s.D, s.Hg, s.Wg, s.d_t, s.d_h, s.d_w,
-                               cap_frames=wl.cap, max_pos_t=f_last + F, theta=s.theta)
+    cache = binding.LayerCache(nb, nh, s.D, s.Hg, s.Wg, s.d_t, s.d_h, s.d_w,
+                               cap_frames=wl.cap, max_pos_t=f_last + F, theta=s.theta,
+                               shard=(sh.b0, sh.h0, s.B, s.H) if strong else None)
     # fill the cache: chunks 0 .. last-1, then the last chunk once
     out = torch.empty(s.B, s.L, s.H, s.D, dtype=torch.bfloat16, device=dev)
     for c in range(wl.chunks):
@@ -269,11 +304,14 @@ def run_ours(args, rank, local_rank, world):
     peaks, peak_src = load_peaks()
     attn_avg = reduce_max(sum(attn_ms) / args.steps, world, dev)
     rope_avg = reduce_max(sum(rope_ms) / args.steps, world, dev)
-    attn_tflops = flops / (attn_avg * 1e-3) / 1e12
-    rope_bytes = wl.rope_bytes(rotate_q=not fq)
+    attn_tflops = flops_rank / (attn_avg * 1e-3) / 1e12
+    rope_bytes = wl.rope_bytes(rotate_q=not fq) * nb * nh // (s.B * s.H)
     rope_gbs = rope_bytes / (rope_avg * 1e-3) / 1e9
-    value = world * flops / (step_ms * 1e-3) / 1e12
+    job_flops = flops if strong else world * flops     # all ranks together
+    value = job_flops / (step_ms * 1e-3) / 1e12
+    e2e_value = job_flops / (e2e_ms * 1e-3) / 1e12
     act_bytes = s.B * s.L * s.H * s.D * 2
+    rope_traffic = profile_traffic(f"rope_kv_append_{wl.name}.txt", ROPE_SOURCES)
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -283,22 +321,13 @@ def run_ours(args, rank, local_rank, world):
         "warmup": args.warmup,
         "ms_per_step": round(step_ms, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if strong else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) fp32 draws rounded to bf16 (q, k, v)",
-        "config": {
-            "workload": f"{wl.name}: B={s.B} H={s.H} D={s.D} grid={s.Hg}x{s.Wg} "
-                        f"L={s.L} keys={Lk} window={wl.window} cap={wl.cap}",
-            "per_rank": "one independent stream per GPU" if world > 1 else "one stream",
-            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, then "
-                  f"{L2_FLUSH_BYTES >> 20} MiB read)",
-            "parallelism": f"independent streams x{world}",
-            "q_rope": "in the attention prologue (append moves k, v only)" if fq else
-                      "in the append (q rotated in place)",
-        },
-        "chunk_steps_per_s": round(world * s.B / (step_ms * 1e-3), 2),
-        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "config": arm_config(wl, world, args),
+        "chunk_steps_per_s": round((1 if strong else world) * s.B / (step_ms * 1e-3), 2),
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
                 "h2d_bytes_per_step": 3 * act_bytes, "d2h_bytes_per_step": act_bytes,
                 "how": "pinned host q/k/v -> device, both calls, device -> pinned host out, "
@@ -314,10 +343,9 @@ def run_ours(args, rank, local_rank, world):
             "peak_source": f"{peak_src} bf16 burst",
             "unit": "TFLOP/s",
             "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
-            "frac_of_sustained": round(attn_tflops / peaks["bf16_tflops_sustained"], 4),
             "traffic": profiled_traffic(wl.name, rope_q=fq),
             "ms_per_launch": round(attn_avg, 4),
-            "flops_per_launch": flops,
+            "flops_per_launch": flops_rank,
         },
         "rope_roofline": {
             "kernel": f"rope_kv_append_kernel<{s.D}, {str(not fq).lower()}>",
@@ -329,6 +357,11 @@ def run_ours(args, rank, local_rank, world):
             "frac": round(rope_gbs / peaks["hbm_gbs"], 4),
             "bytes_per_launch": rope_bytes,
             "us_per_launch": round(rope_avg * 1e3, 2),
+            # DRAM bytes of one launch from the committed ncu capture, and the rate DRAM itself
+            # sees during the launch (the cache writes mostly stay in L2 until later kernels)
+            "traffic": rope_traffic,
+            "dram_gbs": None if rope_traffic is None else
+            round(rope_traffic / (rope_avg * 1e-3) / 1e9, 1),
         },
         "clocks": clocks,
     }
@@ -414,24 +447,31 @@ def run_reference(args, rank, world):
     for i in range(args.warmup):
         _oracle_sample(wl, qb, kb, vb, [i % s.H], args.ref_rows, seed=i)
     total = 0.0
+    measured = 0.0
     sample = ""
     for i in range(args.steps):
-        step_s, _, sample = _oracle_sample(wl, qb, kb, vb, [i % s.H], args.ref_rows, seed=i)
+        step_s, meas_s, sample = _oracle_sample(wl, qb, kb, vb, [i % s.H], args.ref_rows,
+                                                seed=i)
         total += step_s
+        measured += meas_s
     step_s = total / args.steps
     flops = wl.attn_flops(wl.chunks - 1)
     value = flops / step_s / 1e12
     result = {
         "metric": METRIC, "impl": "reference", "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        # a full step of the fp64 oracle takes minutes: every step runs a bounded sample and
+        # its time is scaled up to the whole step; ms_per_step is that extrapolated figure and
+        # seconds_measured the wall time the timed samples actually took
+        "ms_per_step": round(step_s * 1e3, 3), "extrapolated": True,
+        "seconds_measured": round(measured, 3),
+        "ms_per_step_measured": round(measured / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "strong" if args.scaling == "strong" else "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic: seeded N(0,1) bf16",
-        "config": {"workload": f"{wl.name}: B={s.B} H={s.H} D={s.D} grid={s.Hg}x{s.Wg} "
-                               f"L={s.L} keys={wl.keys_for_chunk(wl.chunks - 1)} "
-                               f"window={wl.window} cap={wl.cap}"},
+        "config": arm_config(wl, world, args),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
                          "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": "per step: " + sample},
+                         "sample": "per step: " + sample + " (extrapolated)"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -674,6 +714,20 @@ def run_clip(args, rank, local_rank, world):
         "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "clocks": clocks}), flush=True)
 
 
+def launch_ranks(n: int, argv, port: int = 0) -> int:
+    """Run this script as ``n`` ranks under torch.distributed.run on 127.0.0.1 (one process
+    per GPU), bounded by a timeout; returns the launcher's exit status."""
+    import socket
+    if port == 0:
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+    cmd = ["timeout", "-k", "60", "1800", sys.executable, "-m", "torch.distributed.run",
+           "--nnodes=1", f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -691,7 +745,13 @@ def main():
     ap.add_argument("--q-rope", choices=["append", "attn"], default="append",
                     help="where the queries are rotated: in the append (q in place) or in the "
                          "attention's prologue")
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="weak: every GPU streams its own copy of the workload; strong: the "
+                         "workload's (stream, head) grid is split over the GPUs, streams first")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # started without a launcher: start one rank per GPU and pass on their exit status
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
     rank, local_rank, world = dist_env()
     if world != args.gpus and "WORLD_SIZE" in os.environ:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -25,6 +25,7 @@ UNSTEP_ERR_UNSUPPORTED = -6
 UNSTEP_ERR_CUDA = -7
 UNSTEP_ERR_DEVICE_TIMEOUT = -8
 UNSTEP_ERR_SCRATCH_LIMIT = -9
+UNSTEP_ERR_DEVICE_BOUNDS = -10
 
 UNSTEP_APPEND_DEFER_Q_ROPE = 1   # unstep_rope_kv_append_ex: leave q alone
 UNSTEP_ATTN_ROPE_Q = 1           # unstep_window_attn_ex: q is un-rotated, rotate it in-kernel
@@ -44,6 +45,8 @@ class unstep_cache_t(ctypes.Structure):
         ("frames_written", ctypes.c_int), ("first_frame", ctypes.c_int),
         ("last_chunk_start", ctypes.c_int), ("last_chunk_frames", ctypes.c_int),
         ("initialized", ctypes.c_int),
+        ("act_B", ctypes.c_int), ("act_H", ctypes.c_int),
+        ("b0", ctypes.c_int), ("h0", ctypes.c_int),
     ]
 
 
@@ -95,6 +98,11 @@ _SIGNATURES = {
                               ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                               ctypes.c_void_p], ctypes.c_int),
     "unstep_conv3d_scratch_bytes": ([], ctypes.c_size_t),
+    "unstep_cache_state_bytes": ([ctypes.POINTER(unstep_cache_t)], ctypes.c_size_t),
+    "unstep_cache_save": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p, ctypes.c_size_t,
+                           ctypes.c_void_p], ctypes.c_int),
+    "unstep_cache_restore": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p, ctypes.c_size_t,
+                              ctypes.c_void_p], ctypes.c_int),
     "unstep_get_device_error": ([ctypes.POINTER(unstep_cache_t), ctypes.c_void_p], ctypes.c_int),
     "unstep_selftest_wait_timeout": ([ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p],
                                      ctypes.c_int),
@@ -158,13 +166,18 @@ class LayerCache:
     """One attention layer's ring-buffer KV cache and RoPE tables, in caller-owned torch memory.
 
     All device memory is allocated here by torch; the library only reads and writes it.
+
+    ``shard=(b0, h0, act_B, act_H)`` makes this cache one shard of a larger layer: it holds
+    streams ``b0 .. b0+B-1`` and heads ``h0 .. h0+H-1`` of activations shaped
+    ``[act_B][L][act_H][D]``, and its calls read and write only those rows of q, k, v and out.
     """
 
     def __init__(self, B: int, H: int, D: int, Hg: int, Wg: int, d_t: int, d_h: int, d_w: int,
                  cap_frames: int, max_pos_t: int, theta: float = 10000.0,
                  device: Optional[torch.device] = None,
                  stream: Optional[torch.cuda.Stream] = None,
-                 scratch: Optional[torch.Tensor] = None, use_scratch: bool = True):
+                 scratch: Optional[torch.Tensor] = None, use_scratch: bool = True,
+                 shard: Optional[Tuple[int, int, int, int]] = None):
         L = lib()
         dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                            torch.cuda.current_device())
@@ -172,6 +185,11 @@ class LayerCache:
         c.B, c.H, c.D, c.Hg, c.Wg = B, H, D, Hg, Wg
         c.d_t, c.d_h, c.d_w, c.theta = d_t, d_h, d_w, float(theta)
         c.cap_frames, c.max_pos_t = cap_frames, max_pos_t
+        # an unsharded cache leaves the shard fields at zero (the activations are [B][L][H][D])
+        b0, h0, act_B, act_H = shard if shard is not None else (0, 0, B, H)
+        if shard is not None:
+            c.b0, c.h0, c.act_B, c.act_H = b0, h0, act_B, act_H
+        self.act_B, self.act_H = act_B, act_H
         tab_bytes = L.unstep_cache_table_bytes(ctypes.byref(c))
         if tab_bytes == 0:
             raise UnstepError(UNSTEP_ERR_ARG, "cache shape rejected")
@@ -235,8 +253,9 @@ class LayerCache:
         c = self.c
         if t.dtype != torch.bfloat16:
             raise ValueError(f"{name} must be bfloat16")
-        if tuple(t.shape) != (c.B, L, c.H, c.D):
-            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(c.B, L, c.H, c.D)}")
+        want = (self.act_B, L, self.act_H, c.D)
+        if tuple(t.shape) != want:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want}")
         if t.device != self.device:
             raise ValueError(f"{name} is on {t.device}, the cache on {self.device}")
 
@@ -306,6 +325,30 @@ class LayerCache:
             _check(rc, "unstep_window_attn")
         return out
 
+    # -- checkpoint / resume -----------------------------------------------------------------
+    def state_bytes(self) -> int:
+        return lib().unstep_cache_state_bytes(ctypes.byref(self.c))
+
+    def save_state(self, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """The layer's state (ring K/V rows, slot_frame, metadata) in a pinned host buffer."""
+        buf = torch.empty((self.state_bytes(),), dtype=torch.uint8).pin_memory()
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.device(self.device):
+            _check(lib().unstep_cache_save(ctypes.byref(self.c), buf.data_ptr(), buf.numel(),
+                                           _stream_handle(s)), "unstep_cache_save")
+        s.synchronize()
+        return buf
+
+    def restore_state(self, buf: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+        """Continue the stream a :meth:`save_state` buffer describes (same shape required)."""
+        if buf.device.type != "cpu" or buf.dtype != torch.uint8 or not buf.is_contiguous():
+            raise ValueError("state must be a contiguous uint8 host tensor")
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.device(self.device):
+            _check(lib().unstep_cache_restore(ctypes.byref(self.c), buf.data_ptr(), buf.numel(),
+                                              _stream_handle(s)), "unstep_cache_restore")
+        s.synchronize()     # the host buffer may be reused once the copies have run
+
     def device_error(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         return lib().unstep_get_device_error(ctypes.byref(self.c), _stream_handle(stream))
 
@@ -356,7 +399,8 @@ class HostStepPipeline:
     def _bufs(self, L: int):
         c = self.c
         if not self.sets or self.sets[0]["q"].shape[1] != L:
-            self.sets = [{n: torch.empty((c.B, L, c.H, c.D), dtype=torch.bfloat16,
+            act = (self.cache.act_B, L, self.cache.act_H, c.D)
+            self.sets = [{n: torch.empty(act, dtype=torch.bfloat16,
                                          device=self.device) for n in ("q", "k", "v", "out")}
                          for _ in range(2)]
         return self.sets

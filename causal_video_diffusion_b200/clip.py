@@ -11,7 +11,7 @@ seeded synthetic tensors, generated on the device before the clip runs.
 """
 from __future__ import annotations
 
-from typing import List, Optional
+from typing import Callable, List, Optional
 
 import torch
 
@@ -70,7 +70,8 @@ class ClipDriver:
         for c in self.caches:
             c.reset(stream=stream)
 
-    def _issue(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+    def _issue(self, stream: Optional[torch.cuda.Stream] = None,
+               on_forward: Optional[Callable[[int], None]] = None) -> None:
         F = self.shape.chunk_frames
         for n, f in enumerate(self.sched):
             f0 = self.wl.frame_idx(f.chunk)
@@ -79,10 +80,13 @@ class ClipDriver:
                 cache.rope_kv_append(q, k, v, f0, F, stream=stream)
                 cache.window_attn(q, self.wl.window, out=self.outs[layer], stream=stream)
             binding.renoise(self.x_hat, self.eps[n], f.next_sigma, out=self.latent, stream=stream)
+            if on_forward is not None:
+                on_forward(n)
 
-    def run(self) -> None:
-        """One clip, eagerly (each call launched from the host as it comes)."""
-        self._issue()
+    def run(self, on_forward: Optional[Callable[[int], None]] = None) -> None:
+        """One clip, eagerly (each call launched from the host as it comes).  ``on_forward(n)``
+        runs on the host after forward n's calls are enqueued (e.g. to copy its outputs)."""
+        self._issue(on_forward=on_forward)
 
     def capture(self) -> torch.cuda.CUDAGraph:
         """Capture one clip as a CUDA graph (call reset() before replaying it)."""

@@ -4,6 +4,7 @@
 // UnStep paper (arXiv 2609.32518), abstract: RoPE from precomputed coefficients, KV indexing and
 // a limited temporal window of the attention KV cache; Table 3: chunks of three latent frames.
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -25,6 +26,10 @@ constexpr int kInitMagic = 0x55535450;  // "USTP"
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Stream and head extents of the activation tensors the cache's shard lives in.
+int act_B(const unstep_cache_t *c) { return c->act_B > 0 ? c->act_B : c->B; }
+int act_H(const unstep_cache_t *c) { return c->act_H > 0 ? c->act_H : c->H; }
+
 // Shape fields only (no pointers): 0 if valid, else a status code.
 int check_shape(const unstep_cache_t *c) {
   if (!c) return UNSTEP_ERR_ARG;
@@ -42,6 +47,12 @@ int check_shape(const unstep_cache_t *c) {
   if (tf > (1ll << 24) || rows > (1ll << 30) || static_cast<long long>(c->B) * c->H > (1ll << 30))
     return UNSTEP_ERR_UNSUPPORTED;
   if (c->max_pos_t > (1 << 24)) return UNSTEP_ERR_UNSUPPORTED;
+  // the shard's place in the activations
+  const long long act_b = act_B(c), act_h = act_H(c);
+  if (c->act_B < 0 || c->act_H < 0 || c->b0 < 0 || c->h0 < 0) return UNSTEP_ERR_ARG;
+  if (c->b0 + static_cast<long long>(c->B) > act_b || c->h0 + static_cast<long long>(c->H) > act_h)
+    return UNSTEP_ERR_ARG;
+  if (act_b * act_h > (1ll << 30)) return UNSTEP_ERR_UNSUPPORTED;
   return UNSTEP_OK;
 }
 
@@ -119,6 +130,57 @@ size_t scratch_bytes_for(const unstep_cache_t *c, int sms) {
          2ull * static_cast<size_t>(sms) * unstep::attn_slot_floats(c->D) * sizeof(float);
 }
 
+// ---- checkpoint buffer header (layout documented with unstep_cache_save) ----
+constexpr int kStateMagic = 0x43545355;  // "USTC"
+constexpr int kStateVersion = 1;
+constexpr size_t kStateSlotOffset = 128;
+
+size_t state_header_bytes(const unstep_cache_t *c) {
+  return kStateSlotOffset + ((sizeof(int) * static_cast<size_t>(c->cap_frames) + 15) / 16) * 16;
+}
+
+void put_i32(unsigned char *p, size_t off, int v) { std::memcpy(p + off, &v, sizeof(int)); }
+int get_i32(const unsigned char *p, size_t off) {
+  int v;
+  std::memcpy(&v, p + off, sizeof(int));
+  return v;
+}
+
+void write_state_header(const unstep_cache_t *c, unsigned char *p) {
+  const int f[14] = {c->B,  c->H,          c->D,         c->Hg,  c->Wg,  c->d_t, c->d_h,
+                     c->d_w, c->cap_frames, c->max_pos_t, act_B(c), act_H(c), c->b0, c->h0};
+  put_i32(p, 0, kStateMagic);
+  put_i32(p, 4, kStateVersion);
+  for (int i = 0; i < 14; ++i) put_i32(p, 8 + 4 * i, f[i]);
+  std::memcpy(p + 64, &c->theta, sizeof(double));
+  put_i32(p, 72, c->frames_written);
+  put_i32(p, 76, c->first_frame);
+  put_i32(p, 80, c->last_chunk_start);
+  put_i32(p, 84, c->last_chunk_frames);
+}
+
+int read_state_header(const unsigned char *p, unstep_cache_t *c) {
+  if (get_i32(p, 0) != kStateMagic || get_i32(p, 4) != kStateVersion) return UNSTEP_ERR_ARG;
+  int *f[14] = {&c->B,  &c->H,          &c->D,         &c->Hg,    &c->Wg,    &c->d_t, &c->d_h,
+                &c->d_w, &c->cap_frames, &c->max_pos_t, &c->act_B, &c->act_H, &c->b0,  &c->h0};
+  for (int i = 0; i < 14; ++i) *f[i] = get_i32(p, 8 + 4 * i);
+  std::memcpy(&c->theta, p + 64, sizeof(double));
+  c->frames_written = get_i32(p, 72);
+  c->first_frame = get_i32(p, 76);
+  c->last_chunk_start = get_i32(p, 80);
+  c->last_chunk_frames = get_i32(p, 84);
+  return UNSTEP_OK;
+}
+
+// Shape and shard identical (the metadata may differ).
+bool same_state_shape(const unstep_cache_t *a, const unstep_cache_t *b) {
+  return a->B == b->B && a->H == b->H && a->D == b->D && a->Hg == b->Hg && a->Wg == b->Wg &&
+         a->d_t == b->d_t && a->d_h == b->d_h && a->d_w == b->d_w &&
+         a->cap_frames == b->cap_frames && a->max_pos_t == b->max_pos_t &&
+         act_B(a) == act_B(b) && act_H(a) == act_H(b) && a->b0 == b->b0 && a->h0 == b->h0 &&
+         std::memcmp(&a->theta, &b->theta, sizeof(double)) == 0;
+}
+
 unsigned next_epoch() {
   static std::atomic<unsigned> counter{0};
   return counter.fetch_add(1, std::memory_order_relaxed) % 0xFFFFFFu + 1u;
@@ -128,7 +190,7 @@ unsigned next_epoch() {
 
 extern "C" {
 
-int unstep_version(void) { return 100; }
+int unstep_version(void) { return 101; }
 
 const char *unstep_status_string(int status) {
   switch (status) {
@@ -143,6 +205,8 @@ const char *unstep_status_string(int status) {
     case UNSTEP_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
     case UNSTEP_ERR_SCRATCH_LIMIT:
       return "the call needs more scratch than the library's fixed device buffer holds";
+    case UNSTEP_ERR_DEVICE_BOUNDS:
+      return "a device-side index check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -267,6 +331,10 @@ int unstep_rope_kv_append_ex(void *q, const void *k, const void *v, unstep_cache
   p.tab_w = p.tab_h + static_cast<size_t>(cache->Hg) * (cache->d_h / 2);
   p.B = cache->B;
   p.H = cache->H;
+  p.act_H = act_H(cache);
+  p.b0 = cache->b0;
+  p.h0 = cache->h0;
+  p.sharded = (p.act_H != p.H || p.b0 != 0 || p.h0 != 0) ? 1 : 0;
   p.D = cache->D;
   p.Hg = cache->Hg;
   p.Wg = cache->Wg;
@@ -279,6 +347,9 @@ int unstep_rope_kv_append_ex(void *q, const void *k, const void *v, unstep_cache
   p.frames = grid.frames;
   p.cap = cache->cap_frames;
   p.rows = cache->cap_frames * p.Tf;
+  p.act_B = act_B(cache);
+  p.max_pos_t = cache->max_pos_t;
+  p.dev_error = cache->dev_error;
   if (unstep::launch_rope_kv_append(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
@@ -326,8 +397,16 @@ int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_pl
   return UNSTEP_OK;
 }
 
-int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window, void *out,
-                          unsigned flags, unstep_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// What unstep_window_attn_ex and unstep_window_attn_noalloc share: validation, the window plan,
+// the tensor maps, the persistent schedule and the launch.  `fixed_buffer` selects the scratch:
+// false, the cache's own (cache->attn_scratch, sized at unstep_cache_init; none: one CTA per
+// unit); true, the library's fixed device buffer, whose counters are zeroed on `st` first.
+int window_attn_launch(const void *q, const unstep_cache_t *cache, int window, void *out,
+                       unsigned flags, bool fixed_buffer, cudaStream_t st) {
   int rc = check_ready(cache);
   if (rc) return rc;
   if (flags & ~static_cast<unsigned>(UNSTEP_ATTN_ROPE_Q)) return UNSTEP_ERR_ARG;
@@ -340,14 +419,41 @@ int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window
   const int tf = cache->Hg * cache->Wg;
   const int L = cache->last_chunk_frames * tf;
   const long long R = static_cast<long long>(cache->cap_frames) * tf;
+  const int n_pairs = (L + 255) / 256;
+  // (head, 256-query) units are numbered in int32 by the kernel
+  const long long units = static_cast<long long>(B) * H * n_pairs;
+  if (units > INT_MAX) return fixed_buffer ? UNSTEP_ERR_SCRATCH_LIMIT : UNSTEP_ERR_UNSUPPORTED;
+  const int U = static_cast<int>(units);
+
+  void *scratch = nullptr;
+  size_t counter_bytes = 0;
+  int sms = 0;
+  if (fixed_buffer) {
+    size_t capacity = 0;
+    if (unstep::static_attn_scratch(&scratch, &capacity) != cudaSuccess) {
+      cudaGetLastError();
+      return UNSTEP_ERR_CUDA;
+    }
+    sms = device_sms();
+    if (sms <= 0) return UNSTEP_ERR_CUDA;
+    counter_bytes = unstep::attn_counter_bytes(U);
+    const size_t need = counter_bytes + 2ull * static_cast<size_t>(sms) *
+                                            unstep::attn_slot_floats(D) * sizeof(float);
+    if (need > capacity) return UNSTEP_ERR_SCRATCH_LIMIT;
+  } else if (cache->attn_scratch) {
+    scratch = cache->attn_scratch;
+    counter_bytes = unstep::attn_counter_bytes(max_units(cache));
+    sms = device_sms();
+  }
 
   CUtensorMap tq, tk, tv;
   {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
-                                static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
-    const cuuint64_t str[3] = {static_cast<cuuint64_t>(D) * 2,
-                               static_cast<cuuint64_t>(H) * D * 2,
-                               static_cast<cuuint64_t>(L) * H * D * 2};
+    // the whole activation tensor; the shard's streams and heads are TMA coordinates
+    const cuuint64_t aB = static_cast<cuuint64_t>(act_B(cache));
+    const cuuint64_t aH = static_cast<cuuint64_t>(act_H(cache));
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), aH, static_cast<cuuint64_t>(L), aB};
+    const cuuint64_t str[3] = {static_cast<cuuint64_t>(D) * 2, aH * D * 2,
+                               static_cast<cuuint64_t>(L) * aH * D * 2};
     const cuuint32_t box[4] = {64, 1, 128, 1};
     if (!encode_bf16(&tq, q, 4, dims, str, box)) return UNSTEP_ERR_CUDA;
   }
@@ -365,9 +471,14 @@ int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window
   p.dev_error = cache->dev_error;
   p.B = B;
   p.H = H;
+  p.act_H = act_H(cache);
+  p.act_B = act_B(cache);
+  p.b0 = cache->b0;
+  p.h0 = cache->h0;
   p.L = L;
-  p.n_pairs = (L + 255) / 256;
-  p.n_units = B * H * p.n_pairs;
+  p.rows = static_cast<int>(R);
+  p.n_pairs = n_pairs;
+  p.n_units = U;
   for (int s = 0; s < 2; ++s) {
     p.seg_row[s] = plan.seg_row[s];
     p.seg_len[s] = plan.seg_len[s];
@@ -376,10 +487,8 @@ int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window
   p.n_tiles = p.seg_tiles[0] + p.seg_tiles[1];
   p.div_pairs = unstep::make_fastdiv(static_cast<uint32_t>(p.n_pairs));
   p.div_heads = unstep::make_fastdiv(static_cast<uint32_t>(H));
-  // persistent schedule: whole units in waves of `sms` CTAs, the remainder split along keys
-  const int sms = cache->attn_scratch ? device_sms() : 0;
-  if (cache->attn_scratch && sms > 0) {
-    const int U = p.n_units;
+  if (scratch && sms > 0) {
+    // persistent schedule: whole units in waves of `sms` CTAs, the remainder split along keys
     p.dp_waves = U / sms;
     const int tail = U - p.dp_waves * sms;
     p.u_tail0 = p.dp_waves * sms;
@@ -389,9 +498,8 @@ int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window
     if (gsk > p.w_tail) gsk = p.w_tail;
     p.g_sk = static_cast<int>(gsk);
     p.grid = p.dp_waves > 0 ? sms : p.g_sk;
-    p.counters = static_cast<unsigned *>(cache->attn_scratch);
-    p.slots = reinterpret_cast<float *>(static_cast<char *>(cache->attn_scratch) +
-                                        unstep::attn_counter_bytes(max_units(cache)));
+    p.counters = static_cast<unsigned *>(scratch);
+    p.slots = reinterpret_cast<float *>(static_cast<char *>(scratch) + counter_bytes);
     p.slot_floats = static_cast<int>(unstep::attn_slot_floats(D));
     p.epoch = next_epoch();
   } else {
@@ -426,12 +534,26 @@ int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window
     p.div_tf = unstep::make_fastdiv(static_cast<uint32_t>(tf));
     p.div_wg = unstep::make_fastdiv(static_cast<uint32_t>(cache->Wg));
   }
-  if (unstep::launch_window_attn(D, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess) {
+  // the fixed buffer keeps whatever the previous call left in it: the counts must start at zero
+  if (fixed_buffer && cudaMemsetAsync(scratch, 0, counter_bytes, st) != cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  if (unstep::launch_window_attn(D, tq, tk, tv, p, st) != cudaSuccess) {
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
   }
   return UNSTEP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int unstep_window_attn_ex(const void *q, const unstep_cache_t *cache, int window, void *out,
+                          unsigned flags, unstep_stream_t stream) {
+  return window_attn_launch(q, cache, window, out, flags, false,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, void *out,
@@ -441,95 +563,8 @@ int unstep_window_attn(const void *q, const unstep_cache_t *cache, int window, v
 
 int unstep_window_attn_noalloc(const void *q, const unstep_cache_t *cache, int window,
                                void *out, unstep_stream_t stream) {
-  int rc = check_ready(cache);
-  if (rc) return rc;
-  if (!q || !out) return UNSTEP_ERR_ARG;
-  if (!aligned16(q) || !aligned16(out)) return UNSTEP_ERR_ALIGN;
-  unstep_window_plan_t plan;
-  rc = unstep_window_plan(cache, window, &plan);
-  if (rc) return rc;
-  const int D = cache->D, H = cache->H, B = cache->B;
-  const int tf = cache->Hg * cache->Wg;
-  const int L = cache->last_chunk_frames * tf;
-  const long long R = static_cast<long long>(cache->cap_frames) * tf;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-
-  // the library's fixed buffer stands in for cache->attn_scratch (which is ignored here)
-  void *scratch = nullptr;
-  size_t capacity = 0;
-  if (unstep::static_attn_scratch(&scratch, &capacity) != cudaSuccess) {
-    cudaGetLastError();
-    return UNSTEP_ERR_CUDA;
-  }
-  const int sms = device_sms();
-  if (sms <= 0) return UNSTEP_ERR_CUDA;
-  const int n_pairs = (L + 255) / 256;
-  const int U = B * H * n_pairs;
-  const size_t counter_bytes = unstep::attn_counter_bytes(U);
-  const size_t need = counter_bytes + 2ull * static_cast<size_t>(sms) *
-                                          unstep::attn_slot_floats(D) * sizeof(float);
-  if (need > capacity) return UNSTEP_ERR_SCRATCH_LIMIT;
-
-  CUtensorMap tq, tk, tv;
-  {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
-                                static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
-    const cuuint64_t str[3] = {static_cast<cuuint64_t>(D) * 2,
-                               static_cast<cuuint64_t>(H) * D * 2,
-                               static_cast<cuuint64_t>(L) * H * D * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    if (!encode_bf16(&tq, q, 4, dims, str, box)) return UNSTEP_ERR_CUDA;
-  }
-  {
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(R),
-                                static_cast<cuuint64_t>(B) * H};
-    const cuuint64_t str[2] = {static_cast<cuuint64_t>(D) * 2,
-                               static_cast<cuuint64_t>(R) * D * 2};
-    const cuuint32_t box[3] = {64, 128, 1};
-    if (!encode_bf16(&tk, cache->k_cache, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
-    if (!encode_bf16(&tv, cache->v_cache, 3, dims, str, box)) return UNSTEP_ERR_CUDA;
-  }
-  unstep::AttnParams p{};
-  p.out = out;
-  p.dev_error = cache->dev_error;
-  p.B = B;
-  p.H = H;
-  p.L = L;
-  p.n_pairs = n_pairs;
-  p.n_units = U;
-  for (int s = 0; s < 2; ++s) {
-    p.seg_row[s] = plan.seg_row[s];
-    p.seg_len[s] = plan.seg_len[s];
-    p.seg_tiles[s] = (plan.seg_len[s] + 127) / 128;
-  }
-  p.n_tiles = p.seg_tiles[0] + p.seg_tiles[1];
-  p.div_pairs = unstep::make_fastdiv(static_cast<uint32_t>(p.n_pairs));
-  p.div_heads = unstep::make_fastdiv(static_cast<uint32_t>(H));
-  p.scale_log2 = static_cast<float>(1.4426950408889634073599 / std::sqrt(static_cast<double>(D)));
-  p.wait_limit_ns = unstep::kWaitLimitNs;
-  p.dp_waves = U / sms;
-  const int tail = U - p.dp_waves * sms;
-  p.u_tail0 = p.dp_waves * sms;
-  p.w_tail = static_cast<long long>(tail) * p.n_tiles;
-  long long gsk = tail > 0 ? static_cast<long long>(tail) * 8 : 0;
-  if (gsk > sms) gsk = sms;
-  if (gsk > p.w_tail) gsk = p.w_tail;
-  p.g_sk = static_cast<int>(gsk);
-  p.grid = p.dp_waves > 0 ? sms : p.g_sk;
-  p.counters = static_cast<unsigned *>(scratch);
-  p.slots = reinterpret_cast<float *>(static_cast<char *>(scratch) + counter_bytes);
-  p.slot_floats = static_cast<int>(unstep::attn_slot_floats(D));
-  p.epoch = next_epoch();
-  // the buffer keeps whatever the previous call left in it: the counts must start at zero
-  if (cudaMemsetAsync(scratch, 0, counter_bytes, st) != cudaSuccess) {
-    cudaGetLastError();
-    return UNSTEP_ERR_CUDA;
-  }
-  if (unstep::launch_window_attn(D, tq, tk, tv, p, st) != cudaSuccess) {
-    cudaGetLastError();
-    return UNSTEP_ERR_CUDA;
-  }
-  return UNSTEP_OK;
+  return window_attn_launch(q, cache, window, out, 0u, true,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int unstep_gemm_bf16(const void *a, int lda, const void *b, int ldb, void *c, int ldc, int M,
@@ -664,6 +699,64 @@ int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *
     cudaGetLastError();
     return UNSTEP_ERR_CUDA;
   }
+  return UNSTEP_OK;
+}
+
+size_t unstep_cache_state_bytes(const unstep_cache_t *cache) {
+  if (check_shape(cache)) return 0;
+  return state_header_bytes(cache) + 2 * unstep_cache_kv_bytes(cache);
+}
+
+int unstep_cache_save(const unstep_cache_t *cache, void *host_dst, size_t bytes,
+                      unstep_stream_t stream) {
+  int rc = check_ready(cache);
+  if (rc) return rc;
+  if (!host_dst || bytes < unstep_cache_state_bytes(cache)) return UNSTEP_ERR_ARG;
+  unsigned char *dst = static_cast<unsigned char *>(host_dst);
+  const size_t hb = state_header_bytes(cache), kvb = unstep_cache_kv_bytes(cache);
+  std::memset(dst, 0, hb);
+  write_state_header(cache, dst);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dst + kStateSlotOffset, cache->slot_frame,
+                      sizeof(int) * cache->cap_frames, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(dst + hb, cache->k_cache, kvb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(dst + hb + kvb, cache->v_cache, kvb, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  return UNSTEP_OK;
+}
+
+int unstep_cache_restore(unstep_cache_t *cache, const void *host_src, size_t bytes,
+                         unstep_stream_t stream) {
+  int rc = check_ready(cache);
+  if (rc) return rc;
+  if (!host_src || bytes < kStateSlotOffset) return UNSTEP_ERR_ARG;
+  const unsigned char *src = static_cast<const unsigned char *>(host_src);
+  unstep_cache_t saved{};
+  rc = read_state_header(src, &saved);
+  if (rc) return rc;
+  if (!same_state_shape(cache, &saved)) return UNSTEP_ERR_SHAPE;
+  if (bytes < unstep_cache_state_bytes(cache)) return UNSTEP_ERR_ARG;
+  // the saved metadata must describe a ring this cache can hold
+  if (saved.last_chunk_frames < 0 || saved.last_chunk_frames > cache->cap_frames ||
+      saved.frames_written < 0 || saved.frames_written > cache->max_pos_t)
+    return UNSTEP_ERR_ARG;
+  const size_t hb = state_header_bytes(cache), kvb = unstep_cache_kv_bytes(cache);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(cache->slot_frame, src + kStateSlotOffset,
+                      sizeof(int) * cache->cap_frames, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(cache->k_cache, src + hb, kvb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(cache->v_cache, src + hb + kvb, kvb, cudaMemcpyHostToDevice, s) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return UNSTEP_ERR_CUDA;
+  }
+  cache->frames_written = saved.frames_written;
+  cache->first_frame = saved.first_frame;
+  cache->last_chunk_start = saved.last_chunk_start;
+  cache->last_chunk_frames = saved.last_chunk_frames;
   return UNSTEP_OK;
 }
 

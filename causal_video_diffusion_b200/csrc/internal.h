@@ -25,6 +25,22 @@ inline FastDiv make_fastdiv(uint32_t d) {
 }
 
 #ifdef __CUDACC__
+// Index checks of the debug build (compiled with -DUNSTEP_DEBUG; empty otherwise): a failed
+// check records UNSTEP_ERR_DEVICE_BOUNDS (-10) in the caller's error word, and the caller skips
+// the access or winds the CTA down through its abort path.  Nothing ever traps.
+#ifdef UNSTEP_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool debug_check(bool ok, int *dev_error) {
+  if (kDebugChecks && !ok) {
+    if (dev_error) atomicCAS(dev_error, 0, -10);
+    return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv &f) {
   return (__umulhi(x, f.m) + x) >> f.l;
 }
@@ -53,10 +69,15 @@ struct RopeAppendParams {
   const float2 *tab_h;  // [Hg][d_h/2]
   const float2 *tab_w;  // [Wg][d_w/2]
   int B, L, H, D;
+  // the shard's place in the activations [.][L][act_H][D]: stream b0 + b, head h0 + h
+  int act_H, b0, h0;
+  int sharded;    // 0: the activations are exactly [B][L][H][D]
   int Hg, Wg, Tf;
   int half_t, half_h, half_w;  // pairs per block
   int frame_idx, frames, cap;
   int rows;       // cap * Tf
+  int act_B, max_pos_t;  // extents the debug build checks indices against
+  int *dev_error;        // where the debug build records a failed check
   int slot0;      // frame_idx mod cap
   int rotate_q;   // 1: q rotated in place; 0: q neither read nor written
   FastDiv div_h;  // by H
@@ -68,9 +89,11 @@ struct RopeAppendParams {
 cudaError_t launch_rope_kv_append(const RopeAppendParams &p, cudaStream_t stream);
 
 struct AttnParams {
-  void *out;         // bf16 [B][L][H][D]
+  void *out;         // bf16 [act_B][L][act_H][D]; the shard's rows are written
   int *dev_error;
-  int B, H, L;
+  int B, H, L;       // the shard: streams and heads of the cache
+  int act_H, b0, h0; // its place in the activations: stream b0 + b, head h0 + h
+  int act_B, rows;   // activation streams and cache rows per (stream, head): debug checks
   int n_pairs;       // units per (b, h): two 128-row query tiles each
   int n_units;       // B * H * n_pairs
   int n_tiles;       // key tiles of 128 rows over both ring segments

@@ -40,15 +40,17 @@ __device__ __forceinline__ uint4 ld_plain(const void *p) {
 }
 
 struct Item {
-  long long e;       // element offset of the 8-channel vector in q/k/v
+  long long e;       // element offset of the 8-channel vector in q/k/v (the activations)
   long long ce;      // element offset in the caches
   float2 cs[4];      // cos/sin of its 4 channel pairs
 };
 
 // Where item `it` (one 8-channel vector of one (stream, token, head)) lives, and its coefficients.
 // All index arithmetic is 32-bit (items < 2^31, checked on the host) with multiply-high division.
+// Returns false only in the debug build, when an index falls outside its tensor (the item is
+// then skipped and the error word set).
 template <int D>
-__device__ __forceinline__ void locate(const RopeAppendParams &p, uint32_t it, Item &m) {
+__device__ __forceinline__ bool locate(const RopeAppendParams &p, uint32_t it, Item &m) {
   constexpr int kLogV = (D == 128) ? 4 : 3;  // 16-byte vectors per head row: D / 8
   const uint32_t c8 = it & ((1u << kLogV) - 1);
   const uint32_t r = it >> kLogV;             // (b*L + l)*H + h
@@ -63,9 +65,21 @@ __device__ __forceinline__ void locate(const RopeAppendParams &p, uint32_t it, I
   const int f = p.frame_idx + static_cast<int>(i);
   int slot = p.slot0 + static_cast<int>(i);   // i < frames <= cap: one wrap at most
   if (slot >= p.cap) slot -= p.cap;
-  m.e = static_cast<long long>(it) * 8;
+  // q, k, v: the shard's stream and head within the activations (it * 8 when unsharded)
+  m.e = p.sharded ? ((static_cast<long long>(p.b0) + b) * p.L + l) * p.act_H * D +
+                        (static_cast<long long>(p.h0) + h) * D + c8 * 8
+                  : static_cast<long long>(it) * 8;
   m.ce = ((static_cast<long long>(b) * p.H + h) * p.rows + static_cast<long long>(slot) * p.Tf +
           tok) * D + c8 * 8;
+  if (kDebugChecks) {
+    const long long n_act = static_cast<long long>(p.act_B) * p.L * p.act_H * D;
+    const long long n_cache = static_cast<long long>(p.B) * p.H * p.rows * D;
+    const bool ok = b < static_cast<uint32_t>(p.B) && h < static_cast<uint32_t>(p.H) &&
+                    i < static_cast<uint32_t>(p.frames) && y < static_cast<uint32_t>(p.Hg) &&
+                    slot >= 0 && slot < p.cap && f >= 0 && f < p.max_pos_t && m.e >= 0 &&
+                    m.e + 8 <= n_act && m.ce >= 0 && m.ce + 8 <= n_cache;
+    if (!debug_check(ok, p.dev_error)) return false;
+  }
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int pr = static_cast<int>(c8) * 4 + u;  // channel pair index
@@ -79,6 +93,7 @@ __device__ __forceinline__ void locate(const RopeAppendParams &p, uint32_t it, I
     }
     m.cs[u] = __ldg(src);
   }
+  return true;
 }
 
 // kQ: q is rotated in place; without it q is neither read nor written.
@@ -89,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
   const uint32_t base = blockIdx.x * (kThreads * kItemsPerThread) + threadIdx.x;
   if (blockIdx.x == 0 && threadIdx.x < p.frames) {
     const int f = p.frame_idx + threadIdx.x;
-    p.slot_frame[f % p.cap] = f;
+    if (debug_check(f >= 0 && p.cap > 0, p.dev_error)) p.slot_frame[f % p.cap] = f;
   }
   Item m[kItemsPerThread];
   uint4 qv[kItemsPerThread], kv[kItemsPerThread], vv[kItemsPerThread];
@@ -97,9 +112,8 @@ __global__ void __launch_bounds__(kThreads) rope_kv_append_kernel(const RopeAppe
 #pragma unroll
   for (int u = 0; u < kItemsPerThread; ++u) {
     const uint32_t it = base + u * kThreads;
-    live[u] = it < n_items;
+    live[u] = it < n_items && locate<D>(p, it, m[u]);
     if (live[u]) {
-      locate<D>(p, it, m[u]);
       if (kQ) qv[u] = ld_plain(static_cast<const __nv_bfloat16 *>(p.q) + m[u].e);
       kv[u] = ld_stream(static_cast<const __nv_bfloat16 *>(p.k) + m[u].e);
       vv[u] = ld_stream(static_cast<const __nv_bfloat16 *>(p.v) + m[u].e);

@@ -60,17 +60,18 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 #ifndef UNSTEP_KV_STAGES
-#define UNSTEP_KV_STAGES 4
+#define UNSTEP_KV_STAGES 2
 #endif
 
 template <int D, bool kRopeQ = false>
 struct Cfg {
   static constexpr int kBoxes = D / 64;                // 128-byte swizzle boxes per row
   static constexpr int kTileBytes = 128 * D * 2;       // 128 rows x D bf16
-  static constexpr int kStages = UNSTEP_KV_STAGES;     // K/V ring stages
+  static constexpr int kStages = UNSTEP_KV_STAGES;     // ring stages, one key tile's K and V each
+  static constexpr int kStageBytes = 2 * kTileBytes;   // K tile, then V tile
   static constexpr int kSmemQ = 0;
   static constexpr int kSmemKV = 2 * kTileBytes;
-  static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
+  static constexpr int kSmemBar = kSmemKV + kStages * kStageBytes;
   static constexpr int kSmemTab = kSmemBar + 256;      // RoPE rows of the chunk (kRopeQ)
   static constexpr int kSmemUsed = kSmemTab + (kRopeQ ? kQRopeTabBytes : 0);
   // at least ~116 KB so that a second CTA (which would block on TMEM) never shares the SM
@@ -506,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
-        int n = 0;   // K/V tiles issued
+        int n = 0;   // key tiles (K/V stages) issued
         int nq = 0;  // Q loads issued
         bool ok = true;
         Seg sg;
@@ -515,26 +516,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q > 0 && !(ok = wait_bounded(q_empty, static_cast<uint32_t>(q - 1) & 1u, g, E)))
             break;
           const int ntq = up.has1 ? 2 : 1;
+          if (kDebugChecks &&
+              !debug_check(up.bh < p.B * p.H && p.b0 + up.b < p.act_B && p.h0 + up.h < p.act_H &&
+                               up.q0 + (ntq - 1) * 128 < p.L && sg.k0 >= 0 && sg.k0 < sg.k1 &&
+                               sg.k1 <= p.n_tiles,
+                           p.dev_error)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(q_full, ntq * C::kTileBytes);
           for (int t = 0; t < ntq; ++t)
             for (int c = 0; c < C::kBoxes; ++c)
               tma_load_4d(smem + C::kSmemQ + t * C::kTileBytes + c * 16384, &tmq, q_full,
-                          c * 64, up.h, up.q0 + t * 128, up.b);
+                          c * 64, p.h0 + up.h, up.q0 + t * 128, p.b0 + up.b);
           nq = q + 1;
           for (int kt = sg.k0; ok && kt < sg.k1; ++kt) {
             int row, valid;
             key_tile(p, kt, row, valid);
-            for (int kv = 0; kv < 2; ++kv) {
-              const int s = n % NS;
-              const uint32_t r = static_cast<uint32_t>(n / NS);
-              if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
-              mbar_arrive_expect_tx(&full[s], C::kTileBytes);
-              const CUtensorMap *m = kv ? &tmv : &tmk;
-              for (int c = 0; c < C::kBoxes; ++c)
-                tma_load_3d(smem + C::kSmemKV + s * C::kTileBytes + c * 16384, m, &full[s],
-                            c * 64, row, up.bh);
-              ++n;
+            if (kDebugChecks &&
+                !debug_check(row >= 0 && row < p.rows && valid >= 1 && valid <= 128,
+                             p.dev_error)) {
+              *abort_flag = 1;
+              ok = false;
+              break;
             }
+            // one stage per key tile: its K tile and its V tile under one barrier
+            const int s = n % NS;
+            const uint32_t r = static_cast<uint32_t>(n / NS);
+            if (!(ok = wait_bounded(&empty[s], (r & 1u) ^ 1u, g, E))) break;
+            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            uint8_t *st = smem + C::kSmemKV + s * C::kStageBytes;
+            for (int c = 0; c < C::kBoxes; ++c)
+              tma_load_3d(st + c * 16384, &tmk, &full[s], c * 64, row, up.bh);
+            for (int c = 0; c < C::kBoxes; ++c)
+              tma_load_3d(st + C::kTileBytes + c * 16384, &tmv, &full[s], c * 64, row, up.bh);
+            ++n;
           }
         }
         if (*abort_flag) {
@@ -558,11 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kHiV = static_cast<uint32_t>(sdesc_sw128(0, 16384, 1024) >> 32);
         const uint32_t loQ = static_cast<uint32_t>(sdesc_sw128(sQ, 16, 1024));
         const uint32_t loK = static_cast<uint32_t>(sdesc_sw128(sKV, 16, 1024));
-        const uint32_t loV = static_cast<uint32_t>(sdesc_sw128(sKV, 16384, 1024));
+        const uint32_t loV =
+            static_cast<uint32_t>(sdesc_sw128(sKV + C::kTileBytes, 16384, 1024));
         auto qk = [&](int t, int s) {
           const uint32_t dS = tmem + (t ? C::kTmS1 : C::kTmS0);
           const uint32_t qa = loQ + static_cast<uint32_t>(t * (C::kTileBytes >> 4));
-          const uint32_t kb = loK + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
+          const uint32_t kb = loK + static_cast<uint32_t>(s * (C::kStageBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = static_cast<uint32_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
@@ -572,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto pv = [&](int t, int s, bool acc) {
           const uint32_t dO = tmem + (t ? C::kTmO1 : C::kTmO0);
           const uint32_t aP = tmem + (t ? C::kTmP1 : C::kTmP0);
-          const uint32_t vb = loV + static_cast<uint32_t>(s * (C::kTileBytes >> 4));
+          const uint32_t vb = loV + static_cast<uint32_t>(s * (C::kStageBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_ts(dO, aP + kk * 8, f2u64(vb + static_cast<uint32_t>(kk * (2048 >> 4)), kHiV),
@@ -581,7 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto wait_full = [&](int k) {
           return wait_bounded(&full[k % NS], static_cast<uint32_t>(k / NS) & 1u, g, E);
         };
-        int n = 0;                  // K/V tiles consumed
+        // Per key tile the issuer waits three times (the next stage, P0, P1) and commits three
+        // times (S0, S1, the stage); o_done is committed only after a segment's last PV, since
+        // the commit that announces S(j) already covers PV(j-1) for a softmax that rescales O.
+        int n = 0;                      // key tiles (stages) consumed
         uint32_t done0 = 0, done1 = 0;  // PVs issued per query tile (barrier phases)
         bool ok = true;
         Seg sg;
@@ -598,41 +619,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             qk(1, n % NS);
             umma_commit(&s_full[1]);
           }
-          umma_commit(&empty[n % NS]);
           if (ntl == 1) umma_commit(q_empty);
           for (int j = 0; j < ntl; ++j) {
-            const int nv = n + 2 * j + 1, nk = n + 2 * j + 2;
+            const int st = (n + j) % NS, nst = (n + j + 1) % NS;
             const bool more = j + 1 < ntl;
-            if (!(ok = wait_full(nv))) break;
             if (!(ok = wait_bounded(&p_ready[0], done0 & 1u, g, E))) break;
             tc_fence_after();
-            pv(0, nv % NS, j > 0);
-            umma_commit(&o_done[0]);
+            pv(0, st, j > 0);
+            if (!more) umma_commit(&o_done[0]);
             ++done0;
             if (more) {
-              if (!(ok = wait_full(nk))) break;
+              if (!(ok = wait_full(n + j + 1))) break;
               tc_fence_after();
-              qk(0, nk % NS);
+              qk(0, nst);
               umma_commit(&s_full[0]);
             }
             if (has1) {
               if (!(ok = wait_bounded(&p_ready[1], done1 & 1u, g, E))) break;
               tc_fence_after();
-              pv(1, nv % NS, j > 0);
-              umma_commit(&o_done[1]);
+              pv(1, st, j > 0);
+              if (!more) umma_commit(&o_done[1]);
               ++done1;
             }
-            umma_commit(&empty[nv % NS]);
+            umma_commit(&empty[st]);  // key tile j's K and V are read for the last time
             if (more) {
               if (has1) {
-                qk(1, nk % NS);
+                qk(1, nst);
                 umma_commit(&s_full[1]);
               }
-              umma_commit(&empty[nk % NS]);
               if (j + 2 == ntl) umma_commit(q_empty);  // the segment's last QK^T is issued
             }
           }
-          n += 2 * ntl;
+          n += ntl;
         }
         // every MMA issued above has completed once `drain` flips
         umma_commit(drain);
@@ -653,6 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale = p.scale_log2;
     constexpr int kTileFloats = D * 128 + 256;  // one query tile of a scratch slot
     uint32_t cnt = 0;                           // key tiles this warpgroup has processed
+    uint32_t n_seg = 0;                         // segments of this query tile completed
     bool ok = true;
     QTabs qt{p.tab_t, p.tab_h, p.tab_w, p.frame0};
     if constexpr (kRopeQ) {
@@ -723,9 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float f = ex2_approx(m_run - m_new);
           l_run *= f;
           m_run = m_new;
-          ok = __all_sync(kFull, wait_bounded(&o_done[i], (cnt - 1) & 1u, g, E));
-          if (!ok) break;
-          tc_fence_after();
+          // PV(j-1) has completed: the commit that announced S(j) was issued after it
 #pragma unroll
           for (int c = 0; c < D / 16; ++c) {
             uint32_t o[16];
@@ -757,11 +774,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&p_ready[i]);
         ++cnt;
       }
-      if (ok) ok = __all_sync(kFull, wait_bounded(&o_done[i], (cnt - 1) & 1u, g, E));
+      // o_done[i] completes once per segment of this query tile, after its last PV
+      if (ok) ok = __all_sync(kFull, wait_bounded(&o_done[i], n_seg & 1u, g, E));
       if (ok) tc_fence_after();
+      ++n_seg;
       const int l = up.q0 + i * 128 + row;
-      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
-                           ((static_cast<long long>(up.b) * p.L + l) * p.H + up.h) * D;
+      if (kDebugChecks &&
+          !debug_check(p.b0 + up.b < p.act_B && p.h0 + up.h < p.act_H &&
+                           (sg.slot < 0 || (sg.slot < 2 * p.grid && 2 * sg.u + i < 2 * p.n_units)),
+                       p.dev_error)) {
+        *abort_flag = 1;
+        ok = false;
+      }
+      __nv_bfloat16 *dst =
+          static_cast<__nv_bfloat16 *>(p.out) +
+          ((static_cast<long long>(p.b0 + up.b) * p.L + l) * p.act_H + p.h0 + up.h) * D;
       if (sg.slot < 0) {
         if (ok) store_row<D>(tO, 1.f / l_run, dst, l < p.L);  // whole unit: normalise, store
         continue;
@@ -794,7 +821,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         merge_word[i] = last;
       }
       wg_sync(i);
-      const bool merge = ok && merge_word[i] != 0;
+      bool merge = ok && merge_word[i] != 0;
+      if (kDebugChecks && merge &&
+          !debug_check(c_first >= 0 && c_first <= c_last && c_last < p.g_sk, p.dev_error)) {
+        *abort_flag = 1;
+        merge = false;
+      }
       wg_sync(i);  // merge_word is rewritten by the next piece
       if (merge) merge_row<D>(p, i, row, t0, c_first, c_last, dst, l < p.L);
     }

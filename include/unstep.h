@@ -56,7 +56,8 @@ enum {
   UNSTEP_ERR_UNSUPPORTED = -6,    /* D not 64/128, or a size beyond the kernels' index range */
   UNSTEP_ERR_CUDA = -7,           /* a CUDA runtime call failed (launch, copy, memset) */
   UNSTEP_ERR_DEVICE_TIMEOUT = -8, /* a kernel gave up waiting (reported by the device word) */
-  UNSTEP_ERR_SCRATCH_LIMIT = -9   /* unstep_window_attn_noalloc: call too large for its buffer */
+  UNSTEP_ERR_SCRATCH_LIMIT = -9,  /* unstep_window_attn_noalloc: call too large for its buffer */
+  UNSTEP_ERR_DEVICE_BOUNDS = -10  /* debug build only: a kernel's index check failed (device word) */
 };
 
 /*
@@ -93,6 +94,15 @@ typedef struct {
   int last_chunk_start;  /* first frame of the latest chunk, -1 before any */
   int last_chunk_frames; /* frames of the latest chunk, 0 before any */
   int initialized;       /* set by unstep_cache_init */
+  /* shard of the activations (caller; all zero = the cache covers the whole activation tensor).
+   * Streams and heads are independent in every step of the layer (the paper's window is per
+   * stream and head), so a layer splits over GPUs by (stream, head) ranges with no exchange.
+   * This cache then holds streams b0 .. b0+B-1 and heads h0 .. h0+H-1 of activations laid out
+   * as [act_B][L][act_H][D]: q, k, v and out are those full tensors, and every call reads and
+   * writes only this shard's rows of them, in place.  act_B = 0 means B, act_H = 0 means H;
+   * 0 <= b0, b0 + B <= act_B, 0 <= h0, h0 + H <= act_H, act_B * act_H <= 2^30. */
+  int act_B, act_H;
+  int b0, h0;
 } unstep_cache_t;
 
 /* The chunk a call covers: `frames` latent frames of Hg x Wg tokens. */
@@ -108,7 +118,7 @@ typedef struct {
   int seg_len[2];              /* rows in each range; seg_len[1] == 0 when the range is one */
 } unstep_window_plan_t;
 
-/* Library version, e.g. 100 for 0.1.0. */
+/* Library version, e.g. 101 for 0.1.1. */
 int unstep_version(void);
 
 /* Text for a status code (static storage). */
@@ -157,6 +167,8 @@ int unstep_append_plan(const unstep_cache_t *cache, int frame_idx, unstep_grid_t
  *   q  : bf16 [B][L][H][D], L = grid.frames*Hg*Wg; rotated IN PLACE.
  *   k  : bf16 [B][L][H][D], read only; its rotation goes to k_cache.
  *   v  : bf16 [B][L][H][D], read only; copied bit-exactly to v_cache.
+ * (For a shard cache, act_B and act_H replace B and H in these layouts and only the shard's
+ * streams and heads are read and written.)
  * Channel pair (2p, 2p+1) of block a (t, h or w, in that channel order) with in-block index j is
  * rotated by +ang, ang = pos_a * theta^(-2j/d_a), pos_t = absolute frame index, pos_h = y,
  * pos_w = x, in fp32 from the fp32 tables, results rounded to bf16 (RNE).  Writes
@@ -200,6 +212,8 @@ int unstep_window_plan(const unstep_cache_t *cache, int window, unstep_window_pl
  *   q   : bf16 [B][L][H][D], the chunk's ROTATED queries (as unstep_rope_kv_append left them),
  *         L = last_chunk_frames*Hg*Wg.
  *   out : bf16 [B][L][H][D]; must not overlap q or the caches.
+ *   (For a shard cache, act_B and act_H replace B and H; only the shard's rows of out are
+ *   written.)
  * out = softmax(q K^T / sqrt(D)) V over the window's keys (unstep_window_plan), every query of
  * the chunk seeing the same keys.  bf16 tensor-core products with fp32 accumulation, fp32
  * online softmax, output rounded to bf16 (RNE).
@@ -317,6 +331,50 @@ int unstep_conv3d_causal(const void *x, const void *w, const float *bias, void *
 /* Bytes of unstep_conv3d_causal's optional scratch on the CURRENT device (it depends on the
  * device's SM count, not on the shape); 0 if the device cannot be queried. */
 size_t unstep_conv3d_scratch_bytes(void);
+
+/*
+ * Checkpoint and resume of a stream's layer state.
+ * A causal video stream is generated chunk by chunk in order (paper, Table 3: seven causal
+ * chunks per clip); between two chunks all the state a layer carries forward is its ring of
+ * K/V rows, slot_frame and the frame-order metadata.  These calls move exactly that state to
+ * and from a host buffer, so that a stream can be paused, moved to another device or process,
+ * and continued with results bit-identical to an uninterrupted run.  The coefficient tables
+ * are not part of the state: they follow from the shape and are rebuilt by unstep_cache_init.
+ *
+ * Buffer layout (byte offsets, all in the host's byte order):
+ *   0   int32 magic "USTC", int32 layout version (1)
+ *   8   int32 B, H, D, Hg, Wg, d_t, d_h, d_w, cap_frames, max_pos_t, act_B, act_H, b0, h0
+ *   64  double theta
+ *   72  int32 frames_written, first_frame, last_chunk_start, last_chunk_frames
+ *   88  (padding to 128)
+ *   128 int32 slot_frame[cap_frames], padded to a multiple of 16 bytes
+ *   then k_cache, then v_cache (unstep_cache_kv_bytes() each, the device layout verbatim)
+ * act_B and act_H are stored as the shard extents in use (B and H when unsharded).
+ */
+
+/* Bytes of a state buffer for this cache's shape (0 if the shape fields are invalid). */
+size_t unstep_cache_state_bytes(const unstep_cache_t *cache);
+
+/*
+ * Enqueue on `stream` the copies of the cache's state into host_dst (bytes >= the state size;
+ * pinned memory lets the copies run asynchronously, pageable memory makes them synchronous).
+ * The buffer is complete once the stream has reached this point: synchronise before reading it.
+ * Errors: ARG (uninitialised cache, NULL buffer, too small), CUDA.
+ */
+int unstep_cache_save(const unstep_cache_t *cache, void *host_dst, size_t bytes,
+                      unstep_stream_t stream);
+
+/*
+ * Restore a state written by unstep_cache_save into an initialised cache of the same shape
+ * (same B, H, D, Hg, Wg, RoPE split, theta, cap_frames, max_pos_t and shard): the K/V rows and
+ * slot_frame are copied to the device on `stream` and the metadata set on the host, so the next
+ * append continues the saved stream.  The host buffer must stay unchanged until the stream has
+ * passed this point.  A buffer whose header does not match is refused before anything is copied.
+ * Errors: ARG (uninitialised cache, NULL or short buffer, bad magic or version), SHAPE (shape
+ * mismatch), CUDA.
+ */
+int unstep_cache_restore(unstep_cache_t *cache, const void *host_src, size_t bytes,
+                         unstep_stream_t stream);
 
 /*
  * Synchronises `stream`, reads *cache->dev_error and returns it (UNSTEP_OK if no kernel reported

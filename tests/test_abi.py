@@ -4,6 +4,7 @@ agrees with the oracle's.  No call here reaches a kernel launch."""
 import ctypes
 import os
 import random
+import struct
 import subprocess
 
 import numpy as np
@@ -52,7 +53,7 @@ def test_status_strings(L):
     for code in range(-8, 1):
         assert L.unstep_status_string(code)
     assert L.unstep_status_string(-8) == b"a device-side wait timed out"
-    assert L.unstep_version() == 100
+    assert L.unstep_version() == 101
 
 
 def test_table_and_cache_sizes(L):
@@ -253,3 +254,72 @@ def test_ex_entry_points_flags_and_errors(L):
     assert L.unstep_rope_kv_append_ex(None, q, q, ctypes.byref(c2), 0, g, defer, None) == \
         B.UNSTEP_ERR_ARG
     assert (c.frames_written, c.last_chunk_start, c.last_chunk_frames) == (6, 3, 3)
+
+
+def test_shard_fields_are_validated_on_the_host(L):
+    """A cache may be a (stream, head) shard of larger activations; the shard must lie inside
+    them (checked with the shape, before any device work)."""
+    s = W.LayerShape(B=2, H=3, D=64, Hg=4, Wg=6, d_t=24, d_h=20, d_w=20)
+    ok = [(0, 0, 0, 0), (0, 0, 2, 3), (1, 2, 3, 5), (0, 0, 2, 0), (0, 9, 0, 12)]
+    bad = [(1, 0, 2, 3), (0, 1, 2, 3), (-1, 0, 3, 3), (0, 0, 1, 3), (0, 0, -1, 3),
+           (0, 0, 1 << 16, 1 << 15)]
+    for fields, want_ok in [(f, True) for f in ok] + [(f, False) for f in bad]:
+        c = _cache(s, 3, max_pos_t=3)
+        c.b0, c.h0, c.act_B, c.act_H = fields
+        assert (L.unstep_cache_table_bytes(ctypes.byref(c)) > 0) == want_ok, fields
+
+
+def _state_header(c, frames_written=6, last=(3, 3)):
+    """A checkpoint header as unstep_cache_save writes it (the layout include/unstep.h gives)."""
+    buf = bytearray(L_state_bytes(c))
+    f = [c.B, c.H, c.D, c.Hg, c.Wg, c.d_t, c.d_h, c.d_w, c.cap_frames, c.max_pos_t,
+         c.act_B or c.B, c.act_H or c.H, c.b0, c.h0]
+    struct.pack_into("<2i14i", buf, 0, 0x43545355, 1, *f)
+    struct.pack_into("<d4i", buf, 64, c.theta, frames_written, 0, last[0], last[1])
+    return buf
+
+
+def L_state_bytes(c):
+    return B.lib().unstep_cache_state_bytes(ctypes.byref(c))
+
+
+def test_state_buffer_size(L):
+    s = W.WORKLOADS["wan_window"].shape
+    c = _cache(s, 9, max_pos_t=21)
+    kv = L.unstep_cache_kv_bytes(ctypes.byref(c))
+    assert kv == s.B * s.H * 9 * s.Hg * s.Wg * s.D * 2
+    # 128-byte header, slot_frame padded to 16 bytes, then K and V
+    assert L.unstep_cache_state_bytes(ctypes.byref(c)) == 128 + 48 + 2 * kv
+    c.B = 0
+    assert L.unstep_cache_state_bytes(ctypes.byref(c)) == 0
+
+
+def test_restore_refuses_foreign_or_damaged_state_before_any_copy(L):
+    """Host-side checks only (the cache's device pointers are fake and never touched)."""
+    s = W.LayerShape(B=1, H=2, D=64, Hg=4, Wg=6, d_t=24, d_h=20, d_w=20)
+    c = _cache(s, 6, max_pos_t=12, fake_ptrs=True)
+    c.initialized = INIT_MAGIC
+    good = _state_header(c)
+    n = len(good)
+
+    def restore(buf, size=None):
+        raw = (ctypes.c_ubyte * len(buf)).from_buffer(buf)
+        return L.unstep_cache_restore(ctypes.byref(c), raw, n if size is None else size, None)
+
+    bad_magic = bytearray(good)
+    bad_magic[0] ^= 1
+    assert restore(bad_magic) == B.UNSTEP_ERR_ARG
+    bad_version = bytearray(good)
+    bad_version[4] = 2
+    assert restore(bad_version) == B.UNSTEP_ERR_ARG
+    for off, val in [(8, 2), (12, 3), (16, 128), (40, 7), (44, 13), (56, 1)]:  # B, H, D, cap, ...
+        other = bytearray(good)
+        other[off:off + 4] = val.to_bytes(4, "little")
+        assert restore(other) == B.UNSTEP_ERR_SHAPE, off
+    theta = bytearray(good)
+    theta[64:72] = struct.pack("<d", 500.0)
+    assert restore(theta) == B.UNSTEP_ERR_SHAPE
+    assert restore(bytearray(good), size=n - 1) == B.UNSTEP_ERR_ARG        # short buffer
+    too_far = _state_header(c, frames_written=13)                          # past max_pos_t
+    assert restore(too_far) == B.UNSTEP_ERR_ARG
+    assert (c.frames_written, c.last_chunk_start) == (0, 0)               # cache unchanged

@@ -30,3 +30,40 @@ def test_source_digest_tracks_the_kernel_files():
     a = bench.source_digest(bench.ATTN_SOURCES)
     assert a == bench.kernel_source_digest()
     assert len({a, bench.source_digest(bench.GEMM_SOURCES), bench.source_digest(bench.CONV_SOURCES)}) == 3
+
+
+def _args(**kw):
+    import argparse
+    d = dict(q_rope="append", scaling="weak", workload="wan_full")
+    d.update(kw)
+    return argparse.Namespace(**d)
+
+
+def test_both_arms_print_the_same_config():
+    """The reference arm (the oracle on the host) describes the workload with the very object
+    the CUDA arm prints, so the two lines are comparable key by key."""
+    from causal_video_diffusion_b200 import workloads as W
+    wl = W.WORKLOADS["wan_full"]
+    for world in (1, 2, 8):
+        for scaling in ("weak", "strong"):
+            a = bench.arm_config(wl, world, _args(scaling=scaling))
+            b = bench.arm_config(wl, world, _args(scaling=scaling))
+            assert a == b
+            assert a["workload"].startswith("wan_full: B=1 H=12 D=128")
+    assert "shards x8" in bench.arm_config(wl, 8, _args(scaling="strong"))["parallelism"]
+    assert "independent" in bench.arm_config(wl, 8, _args())["parallelism"]
+
+
+def test_gpus_flag_starts_its_own_ranks(monkeypatch):
+    """``bench.py --gpus N`` with no launcher environment runs itself as N ranks on 127.0.0.1."""
+    calls = []
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: calls.append(cmd) or 0)
+    assert bench.launch_ranks(4, ["--gpus", "4", "--steps", "3"], port=29512) == 0
+    cmd = calls[0]
+    i = cmd.index("-m")
+    assert cmd[i + 1] == "torch.distributed.run"
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[cmd.index("--master-port") + 1] == "29512"
+    assert cmd[0] == "timeout" and cmd[-3:] == ["--gpus", "4", "--steps", "3"][-3:]
+    assert cmd[-5].endswith("bench.py")

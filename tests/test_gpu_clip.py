@@ -61,3 +61,62 @@ def test_clip_graph_replays_the_eager_clip_exactly():
     want = oracle.renoise(W.bits(drv.x_hat.cpu()), W.bits(drv.eps[-1].cpu()), 0.02)
     got = drv.latent.cpu().double().numpy()
     assert np.max(np.abs(got - want)) < 2e-2
+
+
+def _oracle_clip_check(wl, layers, seed, heads, rows_per_forward=None):
+    """Run the driver eagerly, keep every forward's output of every layer, and recompute each
+    from the oracle with inputs regenerated from the documented seeds (layer, chunk, forward),
+    streamed through one oracle cache per layer in the schedule's order.  This pins the driver's
+    own sequencing: the frame index of every forward, which inputs go to which (forward, layer),
+    and that every layer keeps its own ring."""
+    from causal_video_diffusion_b200 import schedule as S
+    from tests import parity as P
+    s = wl.shape
+    drv = clip.ClipDriver(wl, layers=layers, seed=seed)
+    kept = []
+    drv.run(on_forward=lambda n: kept.append([o.clone() for o in drv.outs]))
+    torch.cuda.synchronize()
+    for c in drv.caches:
+        assert c.device_error() == 0
+    sched = S.clip_schedule("unstep", wl.chunks)
+    assert len(kept) == len(sched) == sum(wl.forwards(c) for c in range(wl.chunks))
+    ols = [P.make_oracle(s, wl.cap, heads=heads) for _ in range(layers)]
+    rng = np.random.default_rng(seed)
+    worst = 0.0
+    for n, f in enumerate(sched):
+        f0 = wl.frame_idx(f.chunk)
+        for layer in range(layers):
+            # drawn again on the device (its generator is the driver's), independently of the
+            # driver's own tensors
+            q, k, v = (t.cpu() for t in W.gen_qkv(W.qkv_seed(seed, layer=layer, chunk=f.chunk,
+                                                               forward=n), s, device="cuda"))
+            q_rot = ols[layer].append(W.bits(q), W.bits(k), W.bits(v), f0, s.chunk_frames)
+            if rows_per_forward is None:
+                rows = [(b, l, h) for b in range(s.B) for h in heads for l in range(s.L)]
+            else:
+                ls = P.sample_rows(s.L, s.Tf, rows_per_forward, rng)
+                rows = [(b, l, h) for b in range(s.B) for h in heads for l in ls]
+            want = ols[layer].attend(q_rot, wl.window, rows)
+            got = kept[n][layer].cpu().double().numpy()
+            g = np.stack([got[b, l, h] for (b, l, h) in rows])
+            e = P.attn_errors(g, want)
+            assert e.max_abs <= P.MAX_ABS and e.mean_abs <= P.MEAN_ABS, (n, layer, e)
+            worst = max(worst, e.max_abs)
+    return worst
+
+
+def test_clip_driver_forwards_match_the_oracle_small_layer():
+    """Every one of the 23 forwards of every layer, all rows and heads, on a small layer that
+    keeps the clip's schedule (seven chunks of three frames, W = 9, the Table 3 forward
+    counts)."""
+    small = W.LayerShape(B=1, H=2, D=64, Hg=6, Wg=8, d_t=24, d_h=20, d_w=20)
+    wl = W.Workload("clip_small", small, cap=9, window=9, chunks=7, layers=2,
+                    forwards_per_chunk=W.WORKLOADS["clip30"].forwards_per_chunk)
+    _oracle_clip_check(wl, layers=2, seed=11, heads=[0, 1])
+
+
+def test_clip_driver_forwards_match_the_oracle_wan_layer():
+    """The Wan-shaped clip on two layers: head 5 of every forward of both layers, on sampled
+    rows (tile and frame boundaries, the partial last tile, random rows)."""
+    _oracle_clip_check(W.WORKLOADS["clip30"], layers=2, seed=12, heads=[5],
+                       rows_per_forward=24)

@@ -58,10 +58,48 @@ def test_noalloc_refuses_calls_beyond_its_buffer():
     cache.rope_kv_append(q, k, v, 0, 3)
     c = cache.c
     saved = (c.B, c.H)
-    c.H = 1 << 20            # pretend a million heads: counters need > 48 MiB
     out = torch.empty_like(q)
-    rc = _noalloc(cache, q, 3, out)
-    c.B, c.H = saved
+    try:
+        c.H = 1 << 20        # pretend a million heads: counters need > 48 MiB
+        rc = _noalloc(cache, q, 3, out)
+    finally:
+        c.B, c.H = saved
     assert rc == binding.UNSTEP_ERR_SCRATCH_LIMIT
     assert binding.lib().unstep_status_string(rc) == (
         b"the call needs more scratch than the library's fixed device buffer holds")
+
+
+@pytest.mark.parametrize("D,split", [(64, (24, 20, 20)), (128, (44, 42, 42))])
+def test_noalloc_limit_is_exact(D, split):
+    """The largest call the buffer holds is accepted and the next larger one is refused.
+
+    The buffer (48 MiB) holds two slots per SM of 2 x (D x 128 + 256) floats and then the
+    counters, 8 bytes per (head, 256-query) unit rounded up to 256 bytes.  With one 72-query
+    chunk every head is one unit, so the head count sets the unit count.  Only the host-side
+    checks run: the cache's K pointer is moved off its 16-byte alignment, so a call that passes
+    the size check stops at the tensor map (UNSTEP_ERR_CUDA) and nothing is ever launched."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    slots = 2 * sms * 2 * (D * 128 + 256) * 4
+    units_max = ((48 << 20) - slots) // 256 * 32
+    shape = W.LayerShape(B=1, H=2, D=D, Hg=4, Wg=6, d_t=split[0], d_h=split[1], d_w=split[2])
+    cache = P.make_cache(shape, 3, max_pos_t=3, use_scratch=False)
+    q, k, v = W.gen_qkv(9, shape, device="cuda")
+    cache.rope_kv_append(q, k, v, 0, 3)
+    torch.cuda.synchronize()
+    c = cache.c
+    saved = (c.H, c.k_cache)
+    out = torch.empty_like(q)
+    try:
+        c.k_cache = c.k_cache + 8
+        c.H = units_max
+        at_limit = _noalloc(cache, q, 3, out)
+        c.H = units_max + 1
+        beyond = _noalloc(cache, q, 3, out)
+    finally:
+        c.H, c.k_cache = saved
+    assert at_limit == binding.UNSTEP_ERR_CUDA, at_limit
+    assert beyond == binding.UNSTEP_ERR_SCRATCH_LIMIT, beyond
+    # the cache is untouched and still works through the regular call
+    want = cache.window_attn(q, 3)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0 and torch.isfinite(want.float()).all()
