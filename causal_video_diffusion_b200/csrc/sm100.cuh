@@ -327,8 +327,8 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 // x = n + f exactly, n = round-to-nearest(x) obtained by adding and subtracting 1.5 * 2^23
 // (fp32 round-to-nearest), f in [-1/2, 1/2]; 2^f is a degree-3 polynomial whose coefficients are
 // the minimax (Remez exchange) fit of the relative error on [-1/2, 1/2] (max relative error
-// 7.5e-5, below bf16's half-ulp 2^-9; see exp2_poly_remez.py beside this file); 2^n is applied by
-// adding n to the exponent field.  Valid for x in [-125, 127]: callers clamp from below, and
+// 7.5e-5, below bf16's half-ulp 2^-9; derived and pinned by tests/exp2_remez.py); 2^n is applied
+// by adding n to the exponent field.  Valid for x in [-125, 127]: callers clamp from below, and
 // x <= 8 here because the running max is never more than 8 below a tile's scores.
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;

@@ -2,7 +2,7 @@
 
 Remez exchange for the degree-3 polynomial p minimising max |p(f) - 2^f| / 2^f on [-1/2, 1/2]:
 solve p(x_i) - 2^x_i = (-1)^i E 2^x_i on n+2 reference points, move the points to the extrema of
-the error, repeat until the error levels.  ``python exp2_poly_remez.py`` prints the coefficients
+the error, repeat until the error levels.  ``python tests/exp2_remez.py`` prints the coefficients
 (float64 and rounded to float32) and the maximum relative error of the fp32 coefficients.
 """
 import numpy as np
