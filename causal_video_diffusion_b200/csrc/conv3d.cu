@@ -99,11 +99,12 @@ __device__ __forceinline__ ConvTile conv_tile(const ConvParams &p, int t, uint32
 // Work list of unit c (a CTA, or a CTA pair walking one list); the grid is persistent.  Without
 // a stream-K tail (g_sk = 0) unit c takes tiles c, c + units, ... whole.  With one, it first takes
 // its share [lo, hi) of the tail tiles' K steps (at most two pieces, as a share is never longer
-// than one tile), then whole tiles w*units + c below tail0.  The tail comes first so that the merges of split tiles overlap the
-// whole tiles' main loops instead of ending the launch.  A piece that is not a whole tile leaves
-// its fp32 sums in the CTA's slot 2 (kCta c + rank) + (piece index); the last of a tile's pieces
-// to finish (an atomic count per tile and rank) adds the others' slots to its own accumulator and
-// stores the tile.  No CTA waits for another.
+// than one tile), then whole tiles w*units + c below tail0.  The tail comes first so that the
+// merges of split tiles overlap the whole tiles' main loops instead of ending the launch.  A
+// piece that is not a whole tile leaves its fp32 sums in the CTA's slot 2 (kCta c + rank) +
+// (piece index); the last of a tile's pieces to finish (an atomic count per tile and rank) sums
+// all the pieces' slots in piece order (so that the result does not depend on which piece
+// finished last) and stores the tile.  No CTA waits for another.
 // ---------------------------------------------------------------------------------------------
 struct ConvItem {
   int t;        // output tile
@@ -498,14 +499,17 @@ __device__ __forceinline__ void conv_body(const CUtensorMap &tmx, const CUtensor
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t o[32];
-        tmem_ld32(src0 + mt * kBN + cc * 32, o);
-        tmem_wait_ld();
         const int nb = c.n0 + cc * 32;
-        if (merge) {
-          // add the other units' pieces of this tile (this CTA's rank)
+        if (!merge) {
+          tmem_ld32(src0 + mt * kBN + cc * 32, o);
+          tmem_wait_ld();
+        } else {
+          // the pieces of this tile (this CTA's rank), its own included, summed in piece order
+          // from the slots: the result does not depend on which piece finished last
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
 #pragma unroll 1
           for (int cp = c_first; cp <= c_last; ++cp) {
-            if (cp == unit) continue;
             const float *other =
                 p.slots +
                 static_cast<long long>(conv_piece_slot<kCta>(p, cp, rank, it.s0)) * kConvSlotFloats;
