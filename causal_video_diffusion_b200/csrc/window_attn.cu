@@ -45,13 +45,14 @@ namespace {
 constexpr int kThreads = 384;
 // Register split: launched at 168 per thread (384 x 168 = 64512), the producer/MMA warpgroup
 // drops to kRegsIo and the two softmax warpgroups rise to kRegsSoftmax; the static_assert keeps
-// 2 x 128 x kRegsSoftmax + 128 x kRegsIo within the launch total (200/96: 63488), so the claim
-// can always be satisfied.
+// 2 x 128 x kRegsSoftmax + 128 x kRegsIo within the launch total (184/128: 63488), so the claim
+// can always be satisfied.  With the polynomial share below, 184/128 measured 1-2 % faster than
+// 200/96 on full-cache and windowed layers.
 #ifndef UNSTEP_REGS_SOFTMAX
-#define UNSTEP_REGS_SOFTMAX 200
+#define UNSTEP_REGS_SOFTMAX 184
 #endif
 #ifndef UNSTEP_REGS_IO
-#define UNSTEP_REGS_IO 96
+#define UNSTEP_REGS_IO 128
 #endif
 constexpr int kRegsSoftmax = UNSTEP_REGS_SOFTMAX;
 constexpr int kRegsIo = UNSTEP_REGS_IO;
@@ -112,8 +113,11 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
 // column pairs of a 128-key tile, the last kEmuPairsPer8 pairs.  MUFU alone (16 per clock per SM)
 // needs as long for one tile's 16384 exponentials as the tensor core needs for the other tile's
 // two 128x128x128 products, so moving part of them to the FMA pipe shortens the softmax phase.
+// The polynomial costs more issue slots than one MUFU op, and the softmax warps share the SM's
+// issue slots with the MMA issuer: 2 of 8 measured fastest (3 of 8: +6 %, 4 of 8: +15 %, 1 of 8
+// and 0 of 8: +2-3 %).
 #ifndef UNSTEP_EMU_PAIRS_PER8
-#define UNSTEP_EMU_PAIRS_PER8 3
+#define UNSTEP_EMU_PAIRS_PER8 2
 #endif
 constexpr int kEmuPairsPer8 = UNSTEP_EMU_PAIRS_PER8;
 
