@@ -592,8 +592,16 @@ int unstep_gemm_bf16(const void *a, int lda, const void *b, int ldb, void *c, in
 #define UNSTEP_GEMM_2SM 1
 #endif
   const bool pair = UNSTEP_GEMM_2SM && M >= 256 && N >= 256;
+  CUtensorMap tc;
+  if (pair) {
+    // the pair kernel stores C through TMA, one 64-column x 32-row box per epilogue warp
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t str[1] = {static_cast<cuuint64_t>(ldc) * 2};
+    const cuuint32_t box[2] = {64, 32};
+    if (!encode_bf16(&tc, c, 2, dims, str, box)) return UNSTEP_ERR_CUDA;
+  }
   const cudaError_t e =
-      pair ? unstep::launch_gemm2sm_bf16_tn(ta, tb, c, M, N, K, ldc, dev_error,
+      pair ? unstep::launch_gemm2sm_bf16_tn(ta, tb, tc, M, N, K, dev_error,
                                             reinterpret_cast<cudaStream_t>(stream))
            : unstep::launch_gemm_bf16_tn(ta, tb, c, M, N, K, ldc, dev_error,
                                          reinterpret_cast<cudaStream_t>(stream));

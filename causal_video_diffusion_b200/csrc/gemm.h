@@ -14,8 +14,10 @@ namespace unstep {
 cudaError_t launch_gemm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
                                 int N, int K, int ldc, int *dev_error, cudaStream_t stream);
 
-// The same product on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles); same tensor maps.
-cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
-                                   int N, int K, int ldc, int *dev_error, cudaStream_t stream);
+// The same product on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles); same A and B
+// tensor maps, and C through tmc: 2D (N, M) box (64, 32), 128B swizzle (row stride ldc * 2).
+cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb,
+                                   const CUtensorMap &tc, int M, int N, int K, int *dev_error,
+                                   cudaStream_t stream);
 
 }  // namespace unstep

@@ -14,9 +14,14 @@
 //   * CTA 0's MMA thread commits to the stage's "empty" barrier and to "acc_full" in both CTAs
 //     (multicast commit), so each producer refills its own stage and each epilogue drains its
 //     own rows;
-//   * each epilogue thread arrives on CTA 0's "acc_empty" (128 local + 128 remote arrivals);
+//   * each epilogue thread arrives on CTA 0's "acc_empty" (128 local + 128 remote arrivals) once
+//     it has read its row of the accumulator out of TMEM;
 //   * TMEM is allocated and freed by warp 1 of both CTAs together; the pair meets at cluster
 //     barriers after set-up and before TMEM is freed.
+// Epilogue: each of the four epilogue warps owns 32 rows; per 64-column chunk it rounds its rows
+// to bf16 into a 4 KB staging buffer in shared memory (the 128-byte-swizzled layout of a 64 x 32
+// TMA box) and one lane stores the box with a bulk tensor copy.  Two buffers per warp alternate,
+// so the rounding of one chunk overlaps the store of the previous one.
 // No TMA load uses multicast.  Every wait is bounded (WaitGuard).
 #include <cuda_bf16.h>
 
@@ -36,8 +41,12 @@ constexpr int kThreads = 256;                    // warp 0 TMA, warp 1 MMA, warp
 constexpr int kABytes = 128 * kBK * 2;           // this CTA's 128 rows of A: 16 KB
 constexpr int kBBytes = 128 * kBK * 2;           // this CTA's 128 rows of B: 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kSmemBar = kStages * kStageBytes;
+constexpr int kOutCols = 64;                     // columns per staged output box
+constexpr int kStgBytes = 32 * kOutCols * 2;     // one warp's 32 rows x 64 columns: 4 KB
+constexpr int kSmemStg = kStages * kStageBytes;  // 2 staging buffers per epilogue warp
+constexpr int kSmemBar = kSmemStg + 4 * 2 * kStgBytes;
 constexpr int kSmemAlloc = kSmemBar + 256 + 1024;
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 constexpr int kAccCols = kTN;                    // 256 TMEM columns per accumulator set
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
@@ -103,6 +112,30 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
                : "memory");
 }
 
+// TMA 2D store of a box from this CTA's shared memory (bulk async-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(smem_u32(src))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Until at most one bulk group of this thread still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Until every bulk group of this thread has completed (its writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return;
   const uint64_t t0 = globaltimer_ns();
@@ -115,8 +148,9 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 // column (tile t -> n block t / m_tiles, m block t % m_tiles).
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm2sm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tma,
-                           const __grid_constant__ CUtensorMap tmb, __nv_bfloat16 *out, int M,
-                           int N, int K, int ldc, int *dev_error, uint64_t wait_limit_ns) {
+                           const __grid_constant__ CUtensorMap tmb,
+                           const __grid_constant__ CUtensorMap tmc, int M, int N, int K,
+                           int *dev_error, uint64_t wait_limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -223,44 +257,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int row = threadIdx.x - 128;  // TMEM lane = this CTA's output row
-    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const int wq = warp - 4;            // this warp's 32 TMEM lanes = output rows 32 wq ..
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t acc_empty0 = peer_addr(&acc_empty[0], 0);
     const uint32_t acc_empty1 = peer_addr(&acc_empty[1], 0);
+    uint8_t *stg = smem + kSmemStg + wq * 2 * kStgBytes;
+    if (lane == 0) tma_prefetch_desc(&tmc);
     bool ok = true;
-    int i = 0;
+    int i = 0, nst = 0;
     for (int t = pair; t < tiles; t += pairs, ++i) {
       const int acc = i & 1;
       if (ok)
         ok = __all_sync(kFull, wait_bounded(&acc_full[acc], static_cast<uint32_t>(i >> 1) & 1u, g, E));
       if (!ok) break;
       tc_fence_after();
-      const int m = (t % m_tiles) * kTM + 128 * static_cast<int>(rank) + row;
+      const int m0 = (t % m_tiles) * kTM + 128 * static_cast<int>(rank) + wq * 32;
       const int n0 = (t / m_tiles) * kTN;
       const uint32_t src = tmem + lane_base + acc * kAccCols;
 #pragma unroll 1
-      for (int c = 0; c < kTN / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(src + c * 32, o);
+      for (int c = 0; c < kTN / kOutCols; ++c, ++nst) {
+        uint32_t o[2][32];
+        tmem_ld32(src + c * kOutCols, o[0]);
+        tmem_ld32(src + c * kOutCols + 32, o[1]);
         tmem_wait_ld();
-        const int nn = n0 + c * 32;
-        if (m < M && nn < N) {
-          uint32_t w[16];
+        uint8_t *buf = stg + (nst & 1) * kStgBytes;
+        if (lane == 0) bulk_wait_read1();  // the store issued from this buffer two chunks ago
+        __syncwarp();
+        // row `lane` of the box: 16-byte chunk j (columns 8j .. 8j+7) at position j ^ (lane & 7)
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
-          __nv_bfloat16 *dst = out + static_cast<long long>(m) * ldc + nn;
-          const int nv = (N - nn) >= 32 ? 4 : (N - nn) / 8;  // 16-byte groups (N % 8 == 0)
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            if (v < nv)
-              reinterpret_cast<uint4 *>(dst)[v] =
-                  make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        for (int j = 0; j < 8; ++j) {
+          const int h = j >> 2, e = (j & 3) * 8;
+          const uint4 v = make_uint4(
+              pack_bf16x2(__uint_as_float(o[h][e]), __uint_as_float(o[h][e + 1])),
+              pack_bf16x2(__uint_as_float(o[h][e + 2]), __uint_as_float(o[h][e + 3])),
+              pack_bf16x2(__uint_as_float(o[h][e + 4]), __uint_as_float(o[h][e + 5])),
+              pack_bf16x2(__uint_as_float(o[h][e + 6]), __uint_as_float(o[h][e + 7])));
+          *reinterpret_cast<uint4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past M and columns past N are clipped by the tensor map; a box that starts
+          // past either edge holds nothing of the output and is not stored
+          if (m0 < M && n0 + c * kOutCols < N) tma_store_2d(&tmc, buf, n0 + c * kOutCols, m0);
+          bulk_commit();
         }
       }
       tc_fence_before();
       mbar_arrive_remote(acc ? acc_empty1 : acc_empty0);
     }
+    if (lane == 0) bulk_wait_all();  // the stores have read the buffers and written C
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -276,8 +323,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb, void *c, int M,
-                                   int N, int K, int ldc, int *dev_error, cudaStream_t stream) {
+cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb,
+                                   const CUtensorMap &tc, int M, int N, int K, int *dev_error,
+                                   cudaStream_t stream) {
   static unsigned long long attr_set = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -298,7 +346,7 @@ cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb,
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
   if (pairs < 1) return cudaErrorInvalidConfiguration;
   gemm2sm_bf16_tn_kernel<<<2 * pairs, kThreads, kSmemAlloc, stream>>>(
-      ta, tb, static_cast<__nv_bfloat16 *>(c), M, N, K, ldc, dev_error, kWaitLimitNs);
+      ta, tb, tc, M, N, K, dev_error, kWaitLimitNs);
   return cudaGetLastError();
 }
 
