@@ -22,6 +22,11 @@
 // to bf16 into a 4 KB staging buffer in shared memory (the 128-byte-swizzled layout of a 64 x 32
 // TMA box) and one lane stores the box with a bulk tensor copy.  Two buffers per warp alternate,
 // so the rounding of one chunk overlaps the store of the previous one.
+// Launch overlap: the kernel is launched with programmatic stream serialization and lets its
+// dependents launch as soon as it starts, so that the next product's CTAs set up (barriers, TMEM,
+// cluster sync) on the SMs this grid's finished pairs release; the producer alone waits for the
+// preceding grid (griddepcontrol.wait) before its first load, and everything this grid writes
+// follows that wait.
 // No TMA load uses multicast.  Every wait is bounded (WaitGuard).
 #include <cuda_bf16.h>
 
@@ -33,6 +38,9 @@ namespace unstep {
 namespace {
 
 constexpr int kTM = 256, kTN = 256, kBK = 64;    // output tile of a pair, K step
+#ifndef UNSTEP_GEMM_PDL
+#define UNSTEP_GEMM_PDL 1
+#endif
 #ifndef UNSTEP_GEMM2SM_STAGES
 #define UNSTEP_GEMM2SM_STAGES 6
 #endif
@@ -151,6 +159,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tmb,
                            const __grid_constant__ CUtensorMap tmc, int M, int N, int K,
                            int *dev_error, uint64_t wait_limit_ns) {
+  if (UNSTEP_GEMM_PDL && threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -202,6 +211,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tma);
       tma_prefetch_desc(&tmb);
+      // A and B may be the preceding grid's output: wait for it to complete before any load
+      if (UNSTEP_GEMM_PDL) asm volatile("griddepcontrol.wait;" ::: "memory");
       int n = 0;  // stage fills issued
       bool ok = true;
       for (int t = pair; ok && t < tiles; t += pairs) {
@@ -345,8 +356,19 @@ cudaError_t launch_gemm2sm_bf16_tn(const CUtensorMap &ta, const CUtensorMap &tb,
   const int pairs_max = sms / 2;
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
   if (pairs < 1) return cudaErrorInvalidConfiguration;
-  gemm2sm_bf16_tn_kernel<<<2 * pairs, kThreads, kSmemAlloc, stream>>>(
-      ta, tb, tc, M, N, K, dev_error, kWaitLimitNs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = UNSTEP_GEMM_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm2sm_bf16_tn_kernel, ta, tb, tc, M, N, K, dev_error,
+                         kWaitLimitNs);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
