@@ -77,3 +77,46 @@ def test_gemm_deterministic_and_no_device_error():
     torch.cuda.synchronize()
     assert torch.equal(c1, c2)
     assert int(err.item()) == 0
+
+
+def test_back_to_back_products_equal_serialised_ones():
+    """Pair-GEMM launches overlap their set-up with the preceding launch (programmatic dependent
+    launch): a chain in which every product reads the previous one's output (read after write)
+    and overwrites a buffer the previous one read (write after read), issued back to back on one
+    stream, must give the bits of the same chain with the device synchronised between calls."""
+    M, d, r = 4680, 1536, 1472
+    x = W.gen_act(31, M, d).cuda()
+    w = [W.gen_act(32 + i, r if i % 2 == 0 else d, d if i % 2 == 0 else r).cuda()
+         for i in range(4)]
+
+    def chain(sync):
+        t = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        z = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):  # junk in every buffer, so that a read before the write shows
+            t.fill_(7.0); y.fill_(-3.0); z.fill_(5.0)
+            torch.cuda.synchronize()
+        binding.gemm_bf16(x, w[0], t)          # t = x w0^T
+        if sync: torch.cuda.synchronize()
+        binding.gemm_bf16(t, w[1], y)          # y = t w1^T          (reads t)
+        if sync: torch.cuda.synchronize()
+        binding.gemm_bf16(y, w[2], t)          # t = y w2^T          (overwrites what the last read)
+        if sync: torch.cuda.synchronize()
+        binding.gemm_bf16(t, w[3], z)          # z = t w3^T
+        if sync: torch.cuda.synchronize()
+        binding.gemm_bf16(z, w[2], t)          # t = z w2^T
+        torch.cuda.synchronize()
+        return [W.bits(v.cpu()) for v in (t, y, z)]
+
+    want = chain(True)
+    for _ in range(3):
+        got = chain(False)
+        for g, e in zip(got, want):
+            assert np.array_equal(g, e)
+    # and the chain's first product is the oracle's
+    t0 = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+    binding.gemm_bf16(x, w[0], t0)
+    rows = np.arange(0, M, 97)
+    want0 = oracle.matmul_bt(W.bits(x.cpu())[rows], W.bits(w[0].cpu()))
+    mx, mean = _rel_errors(t0.cpu()[rows].double().numpy(), want0)
+    assert mx < 3e-2 and mean < 2e-3
