@@ -120,3 +120,24 @@ def test_back_to_back_products_equal_serialised_ones():
     want0 = oracle.matmul_bt(W.bits(x.cpu())[rows], W.bits(w[0].cpu()))
     mx, mean = _rel_errors(t0.cpu()[rows].double().numpy(), want0)
     assert mx < 3e-2 and mean < 2e-3
+
+
+@pytest.mark.parametrize("M,N,K,extra", [(300, 264, 200, 64), (4680, 1472, 1536, 8), (257, 520, 72, 24)])
+def test_gemm_into_a_wider_output_leaves_the_rest_alone(M, N, K, extra):
+    """unstep_gemm_bf16 with ldc > N (C a column block of a wider matrix): the N columns are the
+    product, bit for bit what ldc = N gives, and the columns N .. ldc - 1 keep their values."""
+    import ctypes
+    a = W.gen_act(M + 41, M, K).cuda()
+    b = W.gen_act(N + 43, N, K).cuda()
+    want = binding.gemm_bf16(a, b)
+    ldc = N + extra
+    big = torch.full((M, ldc), 3.0, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = binding.lib().unstep_gemm_bf16(
+        ctypes.c_void_p(a.data_ptr()), K, ctypes.c_void_p(b.data_ptr()), K,
+        ctypes.c_void_p(big.data_ptr()), ldc, M, N, K, ctypes.c_void_p(err.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 0 and int(err.item()) == 0
+    assert torch.equal(big[:, :N], want)
+    assert bool((big[:, N:] == 3.0).all())
