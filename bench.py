@@ -19,6 +19,7 @@ workload instead.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -112,58 +113,90 @@ def profiled_traffic(workload: str, rope_q: bool = False):
     return profile_traffic(name, ATTN_SOURCES)
 
 
-class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+CLOCK_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+CLOCK_INTERVAL_MS = 50
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+def summarize_clocks(lines, t0, t1):
+    """Median SM clock, maximum clock and active throttle reasons of the nvidia-smi samples taken
+    between wall times t0 and t1 (seconds; the timed region), widened by one sampling interval.
+    A region shorter than the interval may hold no sample: then the sample nearest to its middle
+    stands for it, and ``window`` says so."""
+    rows = []
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 10:
+            continue
+        try:
+            t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            rows.append((t, float(parts[2]), float(parts[3]), parts[6:10]))
+        except ValueError:
+            continue
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+    pad = CLOCK_INTERVAL_MS / 1000.0
+    inside = [r for r in rows if t0 - pad <= r[0] <= t1 + pad]
+    window = "timed region"
+    if not inside:
+        mid = 0.5 * (t0 + t1)
+        inside = [min(rows, key=lambda r: abs(r[0] - mid))]
+        window = "nearest sample (timed region shorter than the sampling interval)"
+    reasons = set()
+    for _, _, _, flags in inside:
+        for n, flag in zip(CLOCK_REASONS, flags):
+            if flag.lower().startswith("active"):
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(r[1] for r in inside),
+            "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
+            "samples": len(inside), "window": window,
+            "region_ms": round(1000.0 * (t1 - t0), 1)}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons; only the samples taken while the
+    timed region (begin() .. end()) runs are summarised."""
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = os.path.join("/tmp", f"unstep_clocks_{os.getpid()}.csv")
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(CLOCK_INTERVAL_MS)],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:  # noqa: BLE001
             self.proc = None
 
+    def begin(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        time.sleep(2 * CLOCK_INTERVAL_MS / 1000.0)  # let a sample after the region land
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:  # noqa: BLE001
             self.proc.kill()
         self.fh.close()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
-            except ValueError:
-                continue
+        with open(self.path) as f:
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for _, _, r in rows:
-            for n, flag in zip(names, r[1:]):
-                if flag.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(r[0] for r in rows),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows)}
+        t1 = self.t1 if self.t1 is not None else time.time()
+        t0 = self.t0 if self.t0 is not None else t1
+        return summarize_clocks(lines, t0, t1)
 
 
 # ----------------------------------------------------------------------------------------------
@@ -273,9 +306,11 @@ def run_ours(args, rank, local_rank, world):
         dist.barrier()
     torch.cuda.synchronize()
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler.begin()
     for i in range(args.steps):
         one_step(events[i])
     torch.cuda.synchronize()
+    sampler.end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -516,9 +551,11 @@ def run_lowrank(args, rank, local_rank, world):
     sampler.start()
     time.sleep(0.3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sampler.begin()
     for e in evs:
         step(e)
     torch.cuda.synchronize()
+    sampler.end()
     clocks = sampler.stop()
     if int(err.item()) != 0:
         raise RuntimeError("device error in the projections")
@@ -603,9 +640,11 @@ def run_vae_conv(args, rank, local_rank, world):
     sampler.start()
     time.sleep(0.3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sampler.begin()
     for e in evs:
         step(e)
     torch.cuda.synchronize()
+    sampler.end()
     clocks = sampler.stop()
     if int(err.item()) != 0:
         raise RuntimeError("device error in the convolution")
@@ -681,11 +720,13 @@ def run_clip(args, rank, local_rank, world):
     time.sleep(0.3)
     reps = max(1, min(args.steps, 10))
     e0, e1 = ev(), ev()
+    sampler.begin()
     e0.record()
     for _ in range(reps):
         drv.replay()
     e1.record()
     e1.synchronize()
+    sampler.end()
     clocks = sampler.stop()
     graph_ms = e0.elapsed_time(e1) / reps
     for c in drv.caches:

@@ -67,3 +67,26 @@ def test_gpus_flag_starts_its_own_ranks(monkeypatch):
     assert cmd[cmd.index("--master-port") + 1] == "29512"
     assert cmd[0] == "timeout" and cmd[-3:] == ["--gpus", "4", "--steps", "3"][-3:]
     assert cmd[-5].endswith("bench.py")
+
+
+def test_clock_summary_keeps_only_the_timed_region():
+    """Samples taken before or after the timed region (an idle GPU at its maximum clock) do not
+    enter the summary; a region shorter than the sampling interval is stood for by the nearest
+    sample, and the line says so."""
+    import datetime
+    base = datetime.datetime(2026, 12, 3, 3, 0, 0)
+
+    def row(dt_ms, mhz, cap):
+        ts = (base + datetime.timedelta(milliseconds=dt_ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        flags = "Active" if cap else "Not Active"
+        return f"{ts}, 0, {mhz}, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, {flags}\n"
+
+    lines = [row(0, 1965, False), row(50, 1965, False), row(300, 1770, True), row(350, 1755, True),
+             row(400, 1785, True), row(700, 1965, False), "garbage line\n"]
+    t = base.timestamp()
+    s = bench.summarize_clocks(lines, t + 0.29, t + 0.41)
+    assert s["samples"] == 3 and s["sm_mhz"] == 1770 and s["reasons"] == ["sw_power_cap"]
+    assert s["window"] == "timed region"
+    s = bench.summarize_clocks(lines, t + 0.51, t + 0.52)  # between samples: the nearest one
+    assert s["samples"] == 1 and s["window"].startswith("nearest") and s["sm_mhz"] == 1785
+    assert bench.summarize_clocks(["x\n"], t, t)["reasons"] == ["unsampled"]
