@@ -224,7 +224,7 @@ def arm_config(wl, world, args):
     }
 
 
-def run_ours(args, rank, local_rank, world):
+def run_ours(args, rank, local_rank, world, emit=True):
     import torch
     from causal_video_diffusion_b200 import binding
     from causal_video_diffusion_b200 import workloads as W
@@ -402,12 +402,17 @@ def run_ours(args, rank, local_rank, world):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, q_src, k_src, v_src, cache, args)
+    if (rank == 0 and world == 1 and emit and args.workload == "wan_full"
+            and not args.no_other_workloads):
+        del cache, q_src, k_src, v_src, out
+        result["other_workloads"] = other_workloads(args, local_rank)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
-    if rank == 0:
+    if rank == 0 and emit:
         print(json.dumps(result), flush=True)
+    return result
 
 
 # ----------------------------------------------------------------------------------------------
@@ -513,7 +518,7 @@ def run_reference(args, rank, world):
     print(json.dumps(result), flush=True)
 
 
-def run_lowrank(args, rank, local_rank, world):
+def run_lowrank(args, rank, local_rank, world, emit=True):
     """The truncated-SVD V and O projections of one chunk (4680 tokens, 1536 -> rank 1413
     stored padded to 1472 -> 1536): four tensor-core GEMMs per step."""
     import torch
@@ -564,7 +569,7 @@ def run_lowrank(args, rank, local_rank, world):
     flops = 2 * (2 * M * d * lowrank.retained_rank(d) * 2)
     peaks, src = load_peaks()
     tf = flops / (ms * 1e-3) / 1e12
-    print(json.dumps({
+    result = {
         "metric": "truncated-SVD V/O projection TFLOP/s at Wan-1.3B shape (rank 0.92)",
         "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
@@ -581,8 +586,10 @@ def run_lowrank(args, rank, local_rank, world):
                      "traffic": profile_traffic("gemm_bf16_lowrank_vo.txt", GEMM_SOURCES)},
         "clocks": clocks,
         "cpu_baseline": None if args.no_cpu_baseline else
-        _lowrank_cpu_baseline(x, facs, flops, M)}),
-        flush=True)
+        _lowrank_cpu_baseline(x, facs, flops, M)}
+    if emit:
+        print(json.dumps(result), flush=True)
+    return result
 
 
 def _lowrank_cpu_baseline(x, facs, flops, M, rows=None):
@@ -605,7 +612,7 @@ def _lowrank_cpu_baseline(x, facs, flops, M, rows=None):
             "seconds_measured": round(dt, 3)}
 
 
-def run_vae_conv(args, rank, local_rank, world):
+def run_vae_conv(args, rank, local_rank, world, emit=True):
     """The VAE decoder's causal 3x3x3 convolution at the latent resolution: one 3-frame chunk of
     the 60x104 latent with its 2 history frames, 384 -> 384 channels (channels-last bf16)."""
     import numpy as np
@@ -652,7 +659,7 @@ def run_vae_conv(args, rank, local_rank, world):
     flops = 2 * B * T * H * Wd * C * 27 * C
     peaks, src = load_peaks()
     tf = flops / (ms * 1e-3) / 1e12
-    print(json.dumps({
+    result = {
         "metric": "VAE decoder causal 3x3x3 conv TFLOP/s at the 60x104 latent (384 -> 384)",
         "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
@@ -668,7 +675,10 @@ def run_vae_conv(args, rank, local_rank, world):
                      "traffic": profile_traffic("conv3d_vae_conv.txt", CONV_SOURCES)},
         "clocks": clocks,
         "cpu_baseline": None if args.no_cpu_baseline else
-        _conv_cpu_baseline(x, w, bias, flops, H)}), flush=True)
+        _conv_cpu_baseline(x, w, bias, flops, H)}
+    if emit:
+        print(json.dumps(result), flush=True)
+    return result
 
 
 def _conv_cpu_baseline(x, w, bias, flops, H, rows=None):
@@ -755,6 +765,40 @@ def run_clip(args, rank, local_rank, world):
         "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "clocks": clocks}), flush=True)
 
 
+OTHER_WORKLOADS = ("wan_window", "long_b4", "lowrank_vo", "vae_conv")
+
+
+def other_workloads(args, local_rank):
+    """The other layer configurations and the measured "next" rows, timed in the same process
+    after the full-cache line (20 steps each after 5 warm-up steps, L2 flushed between steps, no
+    CPU baseline), summarised for the default bench line."""
+    import torch
+    out = {}
+    for name in OTHER_WORKLOADS:
+        a = argparse.Namespace(**vars(args))
+        a.workload, a.steps, a.warmup, a.no_cpu_baseline = name, 20, 5, True
+        a.no_other_workloads = True
+        if name == "lowrank_vo":
+            r = run_lowrank(a, 0, local_rank, 1, emit=False)
+        elif name == "vae_conv":
+            r = run_vae_conv(a, 0, local_rank, 1, emit=False)
+        else:
+            r = run_ours(a, 0, local_rank, 1, emit=False)
+        entry = {"workload": r["config"]["workload"], "value": r["value"], "unit": r["unit"],
+                 "ms_per_step": r["ms_per_step"], "steps": r["steps"],
+                 "roofline_frac": r["roofline"]["frac"], "roofline_kernel": r["roofline"]["kernel"],
+                 "traffic": r["roofline"].get("traffic"),
+                 "clocks": {k: r["clocks"].get(k) for k in ("sm_mhz", "reasons", "samples")}}
+        if "rope_roofline" in r:
+            entry["rope_gbs"] = r["rope_roofline"]["achieved"]
+            entry["rope_frac"] = r["rope_roofline"]["frac"]
+        if "chunk_steps_per_s" in r:
+            entry["chunk_steps_per_s"] = r["chunk_steps_per_s"]
+        out[name] = entry
+        torch.cuda.empty_cache()
+    return out
+
+
 def launch_ranks(n: int, argv, port: int = 0) -> int:
     """Run this script as ``n`` ranks under torch.distributed.run on 127.0.0.1 (one process
     per GPU), bounded by a timeout; returns the launcher's exit status."""
@@ -783,6 +827,9 @@ def main():
                     help="oracle rows per head (at most the chunk's queries) of the CPU baseline")
     ap.add_argument("--ref-rows", type=int, default=32, help="oracle rows per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the other workloads' summary that the default full-cache line "
+                         "carries at N = 1")
     ap.add_argument("--q-rope", choices=["append", "attn"], default="append",
                     help="where the queries are rotated: in the append (q in place) or in the "
                          "attention's prologue")
