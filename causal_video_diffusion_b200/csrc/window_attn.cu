@@ -78,6 +78,8 @@ struct Cfg {
   // at least ~116 KB so that a second CTA (which would block on TMEM) never shares the SM
   static constexpr int kSmemAlloc = (kSmemUsed + 1024 > 118 * 1024) ? kSmemUsed + 1024
                                                                     : 118 * 1024;
+  // e.g. three K/V stages of 64 KB beside the 64 KB of Q do not fit (D = 128)
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA: fewer K/V stages");
   static constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO0 = 256, kTmO1 = 256 + D;
   // P (bf16, 64 columns per tile).  tcgen05.mma operations are only guaranteed to execute in
   // issue order when they have the same shape; QK^T (N = 128) may overwrite the S columns
