@@ -73,6 +73,8 @@ def test_tiny_workload(use_scratch):
     (16, 16, 1, 4, 4, 6, 0, 1, 1),    # 256 queries = exactly two tiles, one-frame chunks
     (3, 5, 3, 3, 3, 3, 100, 1, 2),    # tiny frames (15 tokens), late positions
     (11, 23, 3, 9, 9, 3, 0, 1, 2),    # 759 queries: 6 tiles incl. a partial, 1-3 key segments
+    (3, 43, 1, 3, 3, 5, 0, 1, 2),     # 129 tokens a frame: a 1-row second query tile, and every
+                                      # ring segment ends in a key tile with 1 valid key
 ])
 @pytest.mark.parametrize("use_scratch", [True, False])
 def test_streams_match_oracle(D, split, Hg, Wg, frames, cap, window, chunks, start, Bn, H,
