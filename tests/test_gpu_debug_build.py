@@ -70,3 +70,25 @@ def test_debug_build_wan_window_stream(dbg):
 def test_debug_build_reports_its_status_text(dbg):
     assert dbg.lib().unstep_status_string(dbg.UNSTEP_ERR_DEVICE_BOUNDS) == (
         b"a device-side index check failed (debug build)")
+
+
+def test_debug_build_one_valid_key_tiles(dbg):
+    """129 tokens a frame, one-frame chunks over a 3-frame ring: a 1-row second query tile and
+    ring segments that end in key tiles with a single valid key, with every index check on."""
+    shape = W.LayerShape(B=1, H=2, D=128, Hg=3, Wg=43, d_t=44, d_h=42, d_w=42, chunk_frames=1)
+    cap = window = 3
+    cache = dbg.LayerCache(shape.B, shape.H, shape.D, shape.Hg, shape.Wg, shape.d_t, shape.d_h,
+                           shape.d_w, cap_frames=cap, max_pos_t=8, theta=shape.theta)
+    ol = P.make_oracle(shape, cap)
+    for f in range(6):
+        q, k, v = W.gen_qkv(500 + f, shape)
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        cache.rope_kv_append(qd, kd, vd, f, 1)
+        out = cache.window_attn(qd, window)
+        torch.cuda.synchronize()
+        assert cache.device_error() == 0, f
+        q_rot = ol.append(W.bits(q), W.bits(k), W.bits(v), f, 1)
+        want = ol.attend(q_rot, window)
+        want = want.reshape(shape.B, shape.H, shape.L, shape.D).transpose(0, 2, 1, 3)
+        e = P.attn_errors(out.cpu().double().numpy(), want)
+        assert e.ok(), (f, e)

@@ -71,6 +71,7 @@ def test_tiny_fused_matches_two_call_and_oracle(use_scratch):
     (16, 16, 1, 4, 4, 6, 0, 1, 1),    # 256 queries = exactly two tiles, one-frame chunks
     (3, 5, 3, 3, 3, 3, 100, 1, 2),    # 45 queries (less than a tile), late positions
     (11, 23, 3, 9, 9, 3, 0, 1, 2),    # 759 queries: 6 tiles incl. a partial
+    (3, 43, 1, 3, 3, 5, 0, 1, 2),     # 129 queries: the second query tile holds one row
 ])
 @pytest.mark.parametrize("use_scratch", [True, False])
 def test_fused_streams_match_two_call(D, split, Hg, Wg, frames, cap, window, chunks, start, Bn,
