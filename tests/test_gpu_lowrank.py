@@ -23,7 +23,9 @@ def _rel_errors(got, want):
                                    # of each go through both barrier phases
                                    (4096, 4096, 128), (65536, 200, 64),
                                    # CTA pairs with K ending inside a 128- and a 192-deep step
-                                   (512, 512, 200), (300, 264, 1416)])
+                                   (512, 512, 200), (300, 264, 1416),
+                                   # exactly one pair tile; K shorter than one 64-deep step
+                                   (256, 256, 64), (256, 256, 8)])
 def test_gemm_matches_oracle(M, N, K):
     a = W.gen_act(M * 7 + 1, M, K)
     b = W.gen_act(N * 11 + 2, N, K)
