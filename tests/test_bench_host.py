@@ -90,3 +90,41 @@ def test_clock_summary_keeps_only_the_timed_region():
     s = bench.summarize_clocks(lines, t + 0.51, t + 0.52)  # between samples: the nearest one
     assert s["samples"] == 1 and s["window"].startswith("nearest") and s["sm_mhz"] == 1785
     assert bench.summarize_clocks(["x\n"], t, t)["reasons"] == ["unsampled"]
+
+
+def test_other_workloads_summary_on_stub_legs(monkeypatch):
+    """The default line's summary of the other workloads: one entry per leg with its headline
+    fields, the clip run with its own step count, and a failing leg recorded as an error instead
+    of losing the line."""
+    import argparse
+    seen = {}
+
+    def fake(kind):
+        def run(a, rank, local_rank, world, emit=True):
+            assert emit is False and world == 1 and a.no_cpu_baseline and a.no_other_workloads
+            seen[a.workload] = (a.steps, a.warmup)
+            if a.workload == "vae_conv":
+                raise RuntimeError("device error in the convolution")
+            r = {"config": {"workload": a.workload + ": shape"}, "value": 1.0, "unit": "TFLOP/s",
+                 "ms_per_step": 2.0, "steps": a.steps,
+                 "roofline": {"frac": 0.5, "kernel": kind, "traffic": None},
+                 "clocks": {"sm_mhz": 1965.0, "reasons": [], "samples": 2}}
+            if kind == "attn":
+                r["rope_roofline"] = {"achieved": 5000.0, "frac": 0.76}
+                r["chunk_steps_per_s"] = 1234.0
+            return r
+        return run
+
+    monkeypatch.setattr(bench, "run_ours", fake("attn"))
+    monkeypatch.setattr(bench, "run_lowrank", fake("gemm"))
+    monkeypatch.setattr(bench, "run_vae_conv", fake("conv"))
+    monkeypatch.setattr(bench, "run_clip", fake("clip"))
+    args = argparse.Namespace(workload="wan_full", steps=400, warmup=10, no_cpu_baseline=False,
+                              no_other_workloads=False, seed=1, q_rope="append", scaling="weak")
+    out = bench.other_workloads(args, 0)
+    assert list(out) == list(bench.OTHER_WORKLOADS)
+    assert seen["wan_window"] == (20, 5) and seen["clip30"] == (3, 3)
+    assert out["wan_window"]["rope_frac"] == 0.76 and out["wan_window"]["roofline_frac"] == 0.5
+    assert out["lowrank_vo"]["roofline_kernel"] == "gemm" and "rope_frac" not in out["lowrank_vo"]
+    assert out["vae_conv"] == {"error": "RuntimeError: device error in the convolution"}
+    assert args.workload == "wan_full" and args.steps == 400   # the caller's args untouched
